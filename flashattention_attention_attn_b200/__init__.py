@@ -1,0 +1,27 @@
+"""Fused softmax attention for NVIDIA B200 (sm_100a).
+
+Two entry points, both implemented by hand-written CUDA kernels in the
+shared library built from ``csrc/`` (C ABI declared in ``include/attn.h``):
+
+  attn_fwd           dense (causal) prefill with grouped-query heads
+  paged_attn_decode  one-token decode against a paged KV cache, split-KV
+                     with a log-sum-exp merge
+
+The Python functions here only marshal arguments into that library; there is
+no CPU fallback.  Importing the package does not load the library; the first
+call does, and raises if it is missing.
+"""
+
+from . import inputs  # noqa: F401  (seeded synthetic inputs; no arithmetic)
+
+_BINDING_NAMES = {
+    "attn_fwd", "paged_attn_decode", "attn_check_support", "attn_status_string",
+    "attn_read_device_status", "library", "library_path", "AttnError",
+}
+
+
+def __getattr__(name):
+    if name in _BINDING_NAMES:
+        from . import _binding
+        return getattr(_binding, name)
+    raise AttributeError(name)

@@ -1,0 +1,168 @@
+"""Seeded synthetic inputs shared by the tests, the smoke check and the bench.
+
+This module draws random numbers and lays them out; it holds none of the
+attention arithmetic.  Every tensor comes from a CPU ``torch.Generator``
+seeded per workload, drawn as float32 N(0, 1) and rounded to bf16
+(round-to-nearest-even), so the CUDA path and the fp64 oracle see the very
+same values.
+
+Workloads (all Llama3-8B-shaped except the tiny one):
+  tiny_causal        B=1, H=2, T=S=128, d=64, causal; drawn in [B, H, T, d]
+                     and handed to the library as [B, T, H, d]
+  llama3_8b_prefill  B=2, Hq=32, Hkv=8, T=S=512, d=128, causal, [B, T, H, d]
+  paged_decode_b64   B=64 one-token queries, Hq=32, Hkv=8, d=128,
+                     block_size=16, context lengths uniform in [256, 4096],
+                     every sequence's blocks a random permutation of the pool
+  long_decode_131k   B=1, context 131072 (8192 blocks, permuted ids)
+  long_prefill_16k   B=1, Hq=32, Hkv=8, T=S=16384, d=128, causal
+"""
+
+from __future__ import annotations
+
+from dataclasses import dataclass, field
+
+import torch
+
+BF16 = torch.bfloat16
+
+
+@dataclass(frozen=True)
+class PrefillSpec:
+    B: int
+    Hq: int
+    Hkv: int
+    T: int
+    S: int
+    d: int
+    causal: bool = True
+    seed: int = 0
+    drawn_layout: str = "BTHD"  # layout the values are drawn in
+
+    @property
+    def scale(self) -> float:
+        return 1.0 / (self.d ** 0.5)
+
+
+@dataclass(frozen=True)
+class DecodeSpec:
+    B: int
+    Hq: int
+    Hkv: int
+    d: int
+    block_size: int
+    max_blocks: int
+    ctx_lo: int
+    ctx_hi: int
+    seed: int = 0
+    extra_pool_blocks: int = 0  # unused physical blocks added to the pool
+    fixed_lens: tuple = field(default=())
+
+    @property
+    def scale(self) -> float:
+        return 1.0 / (self.d ** 0.5)
+
+
+WORKLOADS = {
+    "tiny_causal": PrefillSpec(B=1, Hq=2, Hkv=2, T=128, S=128, d=64, causal=True, seed=1000,
+                               drawn_layout="BHTD"),
+    "llama3_8b_prefill": PrefillSpec(B=2, Hq=32, Hkv=8, T=512, S=512, d=128, causal=True, seed=1001),
+    "paged_decode_b64": DecodeSpec(B=64, Hq=32, Hkv=8, d=128, block_size=16, max_blocks=256,
+                                   ctx_lo=256, ctx_hi=4096, seed=1002),
+    "long_decode_131k": DecodeSpec(B=1, Hq=32, Hkv=8, d=128, block_size=16, max_blocks=8192,
+                                   ctx_lo=131072, ctx_hi=131072, seed=1003),
+    "long_prefill_16k": PrefillSpec(B=1, Hq=32, Hkv=8, T=16384, S=16384, d=128, causal=True, seed=1004),
+}
+
+
+def _randn_bf16(gen: torch.Generator, shape) -> torch.Tensor:
+    return torch.randn(*shape, generator=gen, dtype=torch.float32).to(BF16)
+
+
+def make_prefill(spec: PrefillSpec, seed: int | None = None):
+    """Q [B,T,Hq,d], K [B,S,Hkv,d], V [B,S,Hkv,d] bf16 CPU tensors, contiguous.
+
+    Values are drawn in the order Q, K, V.  For ``drawn_layout == "BHTD"`` the
+    draw is in [B, H, T, d] order and the result is permuted to [B, T, H, d]
+    (the layout the library takes) before it is returned.
+    """
+    gen = torch.Generator(device="cpu").manual_seed(spec.seed if seed is None else seed)
+    s = spec
+    if s.drawn_layout == "BHTD":
+        q = _randn_bf16(gen, (s.B, s.Hq, s.T, s.d)).permute(0, 2, 1, 3).contiguous()
+        k = _randn_bf16(gen, (s.B, s.Hkv, s.S, s.d)).permute(0, 2, 1, 3).contiguous()
+        v = _randn_bf16(gen, (s.B, s.Hkv, s.S, s.d)).permute(0, 2, 1, 3).contiguous()
+    else:
+        q = _randn_bf16(gen, (s.B, s.T, s.Hq, s.d))
+        k = _randn_bf16(gen, (s.B, s.S, s.Hkv, s.d))
+        v = _randn_bf16(gen, (s.B, s.S, s.Hkv, s.d))
+    return q, k, v
+
+
+@dataclass
+class PagedInputs:
+    q: torch.Tensor            # [B, Hq, d] bf16
+    k_cache: torch.Tensor      # [num_blocks, block_size, Hkv, d] bf16
+    v_cache: torch.Tensor      # [num_blocks, block_size, Hkv, d] bf16
+    block_table: torch.Tensor  # [B, max_blocks] int32, -1 where unused
+    seq_lens: torch.Tensor     # [B] int32
+    block_size: int
+
+    @property
+    def num_blocks(self) -> int:
+        return int(self.k_cache.shape[0])
+
+
+def make_paged(spec: DecodeSpec, seed: int | None = None, seq_lens=None) -> PagedInputs:
+    """Paged decode inputs.
+
+    Draw order: sequence lengths (uniform integers in [ctx_lo, ctx_hi], or
+    ``seq_lens`` / ``spec.fixed_lens`` when given), a random permutation of
+    the physical block ids, then q, the K pool and the V pool.  The pool holds
+    sum(ceil(len / block_size)) blocks (+ ``extra_pool_blocks`` never
+    referenced); the permuted ids are handed out in order, sequence 0 first.
+    Unused block-table entries hold -1.
+    """
+    s = spec
+    gen = torch.Generator(device="cpu").manual_seed(s.seed if seed is None else seed)
+    if seq_lens is not None:
+        lens = torch.as_tensor(list(seq_lens), dtype=torch.int64)
+    elif s.fixed_lens:
+        lens = torch.as_tensor(list(s.fixed_lens), dtype=torch.int64)
+    else:
+        lens = torch.randint(s.ctx_lo, s.ctx_hi + 1, (s.B,), generator=gen, dtype=torch.int64)
+    assert lens.numel() == s.B
+    nblk = [(int(L) + s.block_size - 1) // s.block_size for L in lens]
+    if max(nblk, default=0) > s.max_blocks:
+        raise ValueError("a sequence needs more blocks than max_blocks")
+    pool = sum(nblk) + s.extra_pool_blocks
+    perm = torch.randperm(max(pool, 1), generator=gen)[:pool].to(torch.int32)
+    table = torch.full((s.B, s.max_blocks), -1, dtype=torch.int32)
+    at = 0
+    for b, n in enumerate(nblk):
+        table[b, :n] = perm[at:at + n]
+        at += n
+    q = _randn_bf16(gen, (s.B, s.Hq, s.d))
+    k_cache = _randn_bf16(gen, (max(pool, 1), s.block_size, s.Hkv, s.d))
+    v_cache = _randn_bf16(gen, (max(pool, 1), s.block_size, s.Hkv, s.d))
+    return PagedInputs(q=q, k_cache=k_cache, v_cache=v_cache, block_table=table,
+                       seq_lens=lens.to(torch.int32), block_size=s.block_size)
+
+
+def permute_pool(inp: PagedInputs, seed: int) -> PagedInputs:
+    """The same logical cache stored under another physical-id permutation.
+
+    Physical block p moves to slot perm[p]; the table is rewritten so that
+    every logical position still names the same values.
+    """
+    gen = torch.Generator(device="cpu").manual_seed(seed)
+    nb = inp.num_blocks
+    perm = torch.randperm(nb, generator=gen)
+    k2 = torch.empty_like(inp.k_cache)
+    v2 = torch.empty_like(inp.v_cache)
+    k2[perm] = inp.k_cache
+    v2[perm] = inp.v_cache
+    table = inp.block_table.clone()
+    used = table >= 0
+    table[used] = perm[table[used].long()].to(torch.int32)
+    return PagedInputs(q=inp.q, k_cache=k2, v_cache=v2, block_table=table,
+                       seq_lens=inp.seq_lens, block_size=inp.block_size)

@@ -1,0 +1,9 @@
+"""fp64 CPU oracle (test infrastructure; never used by the product path)."""
+from .fp64_attention import (  # noqa: F401
+    attention,
+    gather_paged_kv,
+    paged_decode,
+    softmax_rows,
+    split_paged_decode,
+    visible_key_count,
+)

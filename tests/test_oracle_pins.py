@@ -1,0 +1,272 @@
+"""Pins for the fp64 oracle: each test checks it against something other
+than itself (closed forms, brute force, invariants the pages fix, a library
+routine), so that a dropped term, a wrong sign or index, or a transposed
+operand in the oracle fails at least one of them."""
+
+import json
+import math
+import os
+from fractions import Fraction
+
+import numpy as np
+import pytest
+import torch
+
+from oracle import fp64_attention as orc
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden", "closed_form_cases.json")
+
+
+def _val(s):
+    s = str(s).strip()
+    if "ln(" in s:
+        coef, _, rest = s.partition("ln(")
+        c = float(Fraction(coef.rstrip("*"))) if coef.strip() else 1.0
+        return c * math.log(float(Fraction(rest.rstrip(")"))))
+    return float(Fraction(s))
+
+
+def _arr(x):
+    if isinstance(x, list):
+        return np.array([_arr(e) for e in x], dtype=np.float64)
+    return _val(x)
+
+
+def _golden():
+    with open(GOLDEN) as f:
+        return json.load(f)
+
+
+@pytest.mark.parametrize("case", _golden()["prefill"], ids=lambda c: c["name"])
+def test_golden_prefill_closed_forms(case):
+    q = _arr(case["q"])[None]
+    k = _arr(case["k"])[None]
+    v = _arr(case["v"])[None]
+    O, LSE = orc.attention(q, k, v, _val(case["scale"]), case["causal"])
+    np.testing.assert_allclose(O[0], _arr(case["O"]), rtol=0, atol=1e-12)
+    np.testing.assert_allclose(LSE[0], _arr(case["LSE"]), rtol=0, atol=1e-12)
+
+
+@pytest.mark.parametrize("case", _golden()["paged"], ids=lambda c: c["name"])
+def test_golden_paged_closed_forms(case):
+    O, LSE = orc.paged_decode(_arr(case["q"]), _arr(case["k_cache"]), _arr(case["v_cache"]),
+                              np.array(case["block_table"]), np.array(case["seq_lens"]),
+                              case["block_size"], _val(case["scale"]))
+    np.testing.assert_allclose(O, _arr(case["O"]), rtol=0, atol=1e-12)
+    np.testing.assert_allclose(LSE, _arr(case["LSE"]), rtol=0, atol=1e-12)
+
+
+def _rand(shape, seed):
+    return np.random.default_rng(seed).standard_normal(shape)
+
+
+def _brute_force(q, k, v, scale, causal):
+    """Independent naive evaluation with Python floats and math.exp."""
+    B, T, Hq, d = q.shape
+    S, Hkv = k.shape[1], k.shape[2]
+    g = Hq // Hkv
+    O = np.zeros((B, T, Hq, d))
+    L = np.full((B, Hq, T), -math.inf)
+    for b in range(B):
+        for h in range(Hq):
+            for i in range(T):
+                js = [j for j in range(S) if (not causal) or j <= i + S - T]
+                if not js:
+                    continue
+                sc = [scale * sum(float(q[b, i, h, c]) * float(k[b, j, h // g, c]) for c in range(d)) for j in js]
+                mx = max(sc)
+                w = [math.exp(x - mx) for x in sc]
+                tot = sum(w)
+                for c in range(d):
+                    O[b, i, h, c] = sum(wj * float(v[b, j, h // g, c]) for wj, j in zip(w, js)) / tot
+                L[b, h, i] = mx + math.log(tot)
+    return O, L
+
+
+@pytest.mark.parametrize("T,S,causal", [(1, 1, True), (5, 5, True), (3, 7, True), (6, 4, True),
+                                        (4, 6, False), (8, 8, False)])
+def test_brute_force_tiny(T, S, causal):
+    q = _rand((2, T, 4, 8), 1)
+    k = _rand((2, S, 2, 8), 2)
+    v = _rand((2, S, 2, 8), 3)
+    O, L = orc.attention(q, k, v, 0.3, causal)
+    Ob, Lb = _brute_force(q, k, v, 0.3, causal)
+    np.testing.assert_allclose(O, Ob, rtol=0, atol=1e-12)
+    np.testing.assert_allclose(L, Lb, rtol=0, atol=1e-12)
+
+
+def test_softmax_rows_sum_to_one_and_respect_mask():
+    s = _rand((64, 40), 4) * 10
+    counts = np.random.default_rng(5).integers(1, 41, 64)
+    P, m, l = orc.softmax_rows(s, counts)
+    np.testing.assert_allclose(P.sum(axis=1), 1.0, rtol=0, atol=1e-12)
+    for r in range(64):
+        assert np.all(P[r, counts[r]:] == 0)
+        assert m[r] == s[r, :counts[r]].max()
+    assert np.all(P >= 0)
+
+
+def test_uniform_scores_give_running_mean():
+    B, T, H, d = 1, 33, 3, 16
+    q = np.zeros((B, T, H, d))
+    k = _rand((B, T, H, d), 6)
+    v = _rand((B, T, H, d), 7)
+    O, L = orc.attention(q, k, v, 0.125, causal=True)
+    cummean = np.cumsum(v, axis=1) / np.arange(1, T + 1)[None, :, None, None]
+    np.testing.assert_allclose(O, cummean, rtol=0, atol=1e-12)
+    np.testing.assert_allclose(L, np.broadcast_to(np.log(np.arange(1, T + 1)), (B, H, T)), atol=1e-12)
+
+
+def test_single_key_returns_its_value():
+    q = _rand((2, 5, 4, 8), 8)
+    k = _rand((2, 1, 2, 8), 9)
+    v = _rand((2, 1, 2, 8), 10)
+    O, L = orc.attention(q, k, v, 0.7, causal=False)
+    for h in range(4):
+        np.testing.assert_array_equal(O[:, :, h], np.broadcast_to(v[:, 0:1, h // 2], (2, 5, 8)))
+        dot = np.einsum("btc,bc->bt", q[:, :, h], k[:, 0, h // 2])
+        np.testing.assert_allclose(L[:, h], 0.7 * dot, rtol=0, atol=1e-12)
+
+
+def test_causal_row0_is_first_value_row():
+    q = _rand((2, 9, 8, 4), 11) * 5
+    k = _rand((2, 9, 2, 4), 12) * 5
+    v = _rand((2, 9, 2, 4), 13)
+    O, _ = orc.attention(q, k, v, 1.0, causal=True)
+    for h in range(8):
+        np.testing.assert_array_equal(O[:, 0, h], v[:, 0, h // 4])
+
+
+def test_shift_of_all_keys_leaves_output_and_shifts_lse():
+    q = _rand((1, 12, 4, 8), 14)
+    k = _rand((1, 12, 2, 8), 15)
+    v = _rand((1, 12, 2, 8), 16)
+    u = _rand((8,), 17)
+    O1, L1 = orc.attention(q, k, v, 0.4, causal=True)
+    O2, L2 = orc.attention(q, k + u, v, 0.4, causal=True)
+    np.testing.assert_allclose(O2, O1, rtol=0, atol=1e-12)
+    shift = 0.4 * np.einsum("bthc,c->bht", q, u)
+    np.testing.assert_allclose(L2, L1 + shift, rtol=0, atol=1e-11)
+
+
+def test_gqa_equals_mha_with_repeated_heads():
+    q = _rand((2, 10, 8, 8), 18)
+    k = _rand((2, 10, 2, 8), 19)
+    v = _rand((2, 10, 2, 8), 20)
+    O1, L1 = orc.attention(q, k, v, 0.35, causal=True)
+    kr = np.repeat(k, 4, axis=2)  # head h -> kv head h // 4
+    vr = np.repeat(v, 4, axis=2)
+    O2, L2 = orc.attention(q, kr, vr, 0.35, causal=True)
+    np.testing.assert_array_equal(O1, O2)
+    np.testing.assert_array_equal(L1, L2)
+
+
+@pytest.mark.parametrize("causal", [True, False])
+def test_matches_torch_sdpa_fp64(causal):
+    """PyTorch's scaled_dot_product_attention (named on the page as the
+    library form of the same computation), fp64 on the CPU, K/V expanded."""
+    B, T, Hq, Hkv, d = 2, 37, 8, 2, 16
+    q = _rand((B, T, Hq, d), 21)
+    k = _rand((B, T, Hkv, d), 22)
+    v = _rand((B, T, Hkv, d), 23)
+    O, _ = orc.attention(q, k, v, 0.25, causal)
+    tq = torch.from_numpy(q).permute(0, 2, 1, 3)
+    tk = torch.from_numpy(np.repeat(k, Hq // Hkv, axis=2)).permute(0, 2, 1, 3)
+    tv = torch.from_numpy(np.repeat(v, Hq // Hkv, axis=2)).permute(0, 2, 1, 3)
+    ref = torch.nn.functional.scaled_dot_product_attention(tq, tk, tv, is_causal=causal, scale=0.25)
+    np.testing.assert_allclose(O, ref.permute(0, 2, 1, 3).numpy(), rtol=0, atol=1e-12)
+
+
+def test_bottom_right_rows_equal_tail_of_square_prefill():
+    """Reading: with T < S, causal rows are the last T rows of a T' = S prefill."""
+    S, T = 20, 6
+    qfull = _rand((1, S, 4, 8), 24)
+    k = _rand((1, S, 2, 8), 25)
+    v = _rand((1, S, 2, 8), 26)
+    Of, Lf = orc.attention(qfull, k, v, 0.3, causal=True)
+    Ot, Lt = orc.attention(qfull[:, S - T:], k, v, 0.3, causal=True)
+    np.testing.assert_array_equal(Ot, Of[:, S - T:])
+    np.testing.assert_array_equal(Lt, Lf[:, :, S - T:])
+
+
+def test_empty_key_set_gives_zero_and_minus_inf():
+    q = _rand((1, 4, 2, 8), 27)
+    k = np.zeros((1, 0, 2, 8))
+    O, L = orc.attention(q, k, k, 0.3, causal=True)
+    assert np.all(O == 0) and np.all(np.isneginf(L))
+    # T > S bottom-right: the first T - S rows see nothing
+    k = _rand((1, 2, 2, 8), 28)
+    O, L = orc.attention(q, k, k, 0.3, causal=True)
+    assert np.all(O[:, :2] == 0) and np.all(np.isneginf(L[:, :, :2]))
+    assert np.all(np.isfinite(L[:, :, 2:]))
+
+
+def _paged_case(seed, B=5, Hq=8, Hkv=2, d=8, bs=4, max_blocks=9, extra=3):
+    rng = np.random.default_rng(seed)
+    lens = rng.integers(0, bs * max_blocks + 1, B)
+    lens[0] = bs * max_blocks  # one full row
+    lens[1] = 0                # one empty sequence
+    nblk = [(int(L) + bs - 1) // bs for L in lens]
+    pool = sum(nblk) + extra
+    perm = rng.permutation(pool)
+    table = -np.ones((B, max_blocks), dtype=np.int32)
+    at = 0
+    for b, n in enumerate(nblk):
+        table[b, :n] = perm[at:at + n]
+        at += n
+    q = rng.standard_normal((B, Hq, d))
+    kc = rng.standard_normal((pool, bs, Hkv, d))
+    vc = rng.standard_normal((pool, bs, Hkv, d))
+    return q, kc, vc, table, lens, bs
+
+
+def test_paged_result_invariant_under_block_permutation():
+    q, kc, vc, table, lens, bs = _paged_case(29)
+    O1, L1 = orc.paged_decode(q, kc, vc, table, lens, bs, 0.3)
+    perm = np.random.default_rng(30).permutation(kc.shape[0])
+    kc2 = np.empty_like(kc)
+    vc2 = np.empty_like(vc)
+    kc2[perm] = kc
+    vc2[perm] = vc
+    t2 = np.where(table >= 0, perm[np.maximum(table, 0)], -1)
+    O2, L2 = orc.paged_decode(q, kc2, vc2, t2, lens, bs, 0.3)
+    np.testing.assert_array_equal(O1, O2)
+    np.testing.assert_array_equal(L1, L2)
+
+
+def test_paged_decode_equals_last_row_of_causal_prefill():
+    q, kc, vc, table, lens, bs = _paged_case(31)
+    O, L = orc.paged_decode(q, kc, vc, table, lens, bs, 0.3)
+    for b in range(len(lens)):
+        n = int(lens[b])
+        if n == 0:
+            assert np.all(O[b] == 0) and np.all(np.isneginf(L[b]))
+            continue
+        # contiguous cache written position by position (independent of the gather)
+        K = np.stack([kc[table[b, p // bs], p % bs] for p in range(n)])[None]
+        V = np.stack([vc[table[b, p // bs], p % bs] for p in range(n)])[None]
+        Q = np.zeros((1, n, q.shape[1], q.shape[2]))
+        Q[0, n - 1] = q[b]
+        Op, Lp = orc.attention(Q, K, V, 0.3, causal=True)
+        np.testing.assert_allclose(O[b], Op[0, n - 1], rtol=0, atol=1e-12)
+        np.testing.assert_allclose(L[b], Lp[0, :, n - 1], rtol=0, atol=1e-12)
+
+
+@pytest.mark.parametrize("splits", [1, 2, 3, 7, 9, 20])
+def test_split_merge_equals_unsplit(splits):
+    q, kc, vc, table, lens, bs = _paged_case(32)
+    O1, L1 = orc.paged_decode(q, kc, vc, table, lens, bs, 0.3)
+    O2, L2 = orc.split_paged_decode(q, kc, vc, table, lens, bs, 0.3, splits)
+    np.testing.assert_allclose(O2, O1, rtol=0, atol=1e-12)
+    np.testing.assert_allclose(L2, L1, rtol=0, atol=1e-12)
+
+
+def test_unused_table_entries_are_never_read():
+    q, kc, vc, table, lens, bs = _paged_case(33)
+    O1, L1 = orc.paged_decode(q, kc, vc, table, lens, bs, 0.3)
+    t2 = table.copy()
+    for b in range(len(lens)):
+        t2[b, (int(lens[b]) + bs - 1) // bs:] = 10 ** 6  # would raise IndexError if read
+    O2, L2 = orc.paged_decode(q, kc, vc, t2, lens, bs, 0.3)
+    np.testing.assert_array_equal(O1, O2)
+    np.testing.assert_array_equal(L1, L2)
