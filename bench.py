@@ -1,0 +1,394 @@
+"""Benchmark of the fused-attention hot path on B200.
+
+One step = one pass of the whole path over one batch of synthetic input:
+  * attn_fwd          Llama3-8B-shaped causal GQA prefill (B=2, Hq=32, Hkv=8,
+                      T=S=512, d=128)
+  * paged_attn_decode one-token decode of 64 sequences against a paged cache
+                      (Hq=32, Hkv=8, d=128, block_size=16, context U[256,4096])
+The metric is the fraction of the B200 roofline the step reaches: the ideal
+step time is prefill FLOPs / measured bf16 tensor peak + decode bytes /
+measured HBM bandwidth, and value = 100 * (sum over ranks of ideal time) /
+(measured step time, max over ranks): percent of one B200's roofline,
+summed over the GPUs of the job.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload step|long]
+
+`--workload long` times the long-context pair (T=S=16384 prefill and a
+131072-token split-KV decode) with the same accounting.  `--impl reference`
+times the fp64 CPU oracle (the only reference implementation there is) on a
+bounded sample of the same step.
+"""
+
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "prefill attn TFLOP/s & paged-decode KV GB/s, % of B200 roofline"
+UNIT = "% of 1xB200 roofline (summed over GPUs)"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+WORKLOAD_SETS = {
+    "step": ("llama3_8b_prefill", "paged_decode_b64"),
+    "long": ("long_prefill_16k", "long_decode_131k"),
+}
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            pk = json.load(f)
+        return {k: float(pk[k]) for k in FALLBACK_PEAKS}, "measured"
+    except Exception:
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+def parse_args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", choices=sorted(WORKLOAD_SETS), default="step")
+    ap.add_argument("--num-splits", type=int, default=0, help="decode splits (0 = library's choice)")
+    ap.add_argument("--e2e-steps", type=int, default=5)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    return ap.parse_args()
+
+
+# --------------------------------------------------------------------------
+# clocks during the timed region (NVML reads only; nothing is changed)
+# --------------------------------------------------------------------------
+class ClockSampler:
+    REASONS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
+               0x8: "hw_slowdown", 0x10: "sync_boost", 0x20: "sw_thermal_slowdown",
+               0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown", 0x100: "display_clock_setting"}
+
+    def __init__(self, device_index: int, period_s: float = 0.01):
+        self.samples = []
+        self.period = period_s
+        self._stop = threading.Event()
+        self._thr = None
+        self.max_mhz = None
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self._nv = pynvml
+            self._h = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
+        except Exception:
+            self._nv = None
+
+    def _run(self):
+        nv = self._nv
+        while not self._stop.is_set():
+            try:
+                mhz = nv.nvmlDeviceGetClockInfo(self._h, nv.NVML_CLOCK_SM)
+                rs = nv.nvmlDeviceGetCurrentClocksEventReasons(self._h)
+                self.samples.append((time.perf_counter(), mhz, rs))
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def start(self):
+        if self._nv is not None:
+            self._thr = threading.Thread(target=self._run, daemon=True)
+            self._thr.start()
+
+    def stop(self):
+        self._stop.set()
+        if self._thr is not None:
+            self._thr.join()
+
+    def summary(self, t0, t1):
+        if self._nv is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvml unavailable"], "samples": 0}
+        inside = [s for s in self.samples if t0 <= s[0] <= t1]
+        use = inside or self.samples
+        mhz = sorted(s[1] for s in use)
+        bits = 0
+        for s in use:
+            bits |= int(s[2])
+        reasons = [name for bit, name in self.REASONS.items() if bits & bit and name != "gpu_idle"]
+        return {"sm_mhz": mhz[len(mhz) // 2] if mhz else None, "sm_max_mhz": self.max_mhz,
+                "reasons": reasons, "samples": len(inside), "samples_total": len(self.samples)}
+
+
+# --------------------------------------------------------------------------
+# CPU baseline: the fp64 oracle on a bounded sample of the same step
+# --------------------------------------------------------------------------
+def cpu_baseline(pname, dname, peaks, seed_offset=0, budget_s=20.0):
+    import numpy as np
+    import torch
+
+    from flashattention_attention_attn_b200 import inputs, workloads
+    from oracle import fp64_attention as orc
+
+    try:
+        from threadpoolctl import threadpool_info
+        cores = max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
+    except Exception:
+        cores = 1
+    ps = inputs.WORKLOADS[pname]
+    ds = inputs.WORKLOADS[dname]
+    q, k, v = inputs.make_prefill(ps, seed=ps.seed + seed_offset)
+    dinp = inputs.make_paged(ds, seed=ds.seed + seed_offset)
+    f = lambda t: t.to(torch.float64).numpy()  # noqa: E731
+    qd, kd, vd = f(q), f(k), f(v)
+    # prefill sample: all heads of batch 0, an evenly spread set of rows
+    T = ps.T
+    rows = list(range(0, T, max(1, T // 64)))
+    t0 = time.perf_counter()
+    orc.attention(qd[:1], kd[:1], vd[:1], ps.scale, ps.causal, rows=rows)
+    tp = time.perf_counter() - t0
+    # cost of a row is proportional to the keys it sees
+    seen = sum(min(ps.S, i + ps.S - ps.T + 1) if ps.causal else ps.S for i in rows)
+    full_pairs = workloads.visible_pairs(ps.T, ps.S, ps.causal) * ps.B
+    t_prefill = tp * full_pairs / max(seen, 1)
+    # decode sample: leading sequences until ~budget/2 spent or 4 sequences
+    lens = dinp.seq_lens.numpy()
+    kc, vc = f(dinp.k_cache), f(dinp.v_cache)
+    qq = f(dinp.q)
+    done_tok, td, nseq = 0, 0.0, 0
+    for b in range(len(lens)):
+        t0 = time.perf_counter()
+        orc.paged_decode(qq[b:b + 1], kc, vc, dinp.block_table.numpy()[b:b + 1], lens[b:b + 1], 16, ds.scale)
+        td += time.perf_counter() - t0
+        done_tok += int(lens[b])
+        nseq += 1
+        if nseq >= 4 or td > budget_s / 2:
+            break
+    t_decode = td * float(lens.sum()) / max(done_tok, 1)
+    flops = workloads.prefill_flops(ps.B, ps.Hq, ps.T, ps.S, ps.d, ps.causal)
+    dbytes = workloads.decode_bytes(lens, ds.Hq, ds.Hkv, ds.d, ds.block_size)
+    ideal = flops / (peaks["bf16_tflops"] * 1e12) + dbytes / (peaks["hbm_gbs"] * 1e9)
+    est = t_prefill + t_decode
+    return {"value": 100.0 * ideal / est, "unit": UNIT, "cores": int(cores), "kind": "oracle",
+            "sample": (f"fp64 oracle: prefill rows {len(rows)}/{T} of batch 0 (all {ps.Hq} heads), "
+                       f"decode {nseq}/{len(lens)} sequences ({done_tok} tokens); time scaled by visible "
+                       f"pairs / tokens to the full step"),
+            "est_step_s": est}
+
+
+# --------------------------------------------------------------------------
+def main():
+    args = parse_args()
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    pname, dname = WORKLOAD_SETS[args.workload]
+    peaks, peak_src = load_peaks()
+
+    if args.impl == "reference":
+        if rank != 0:
+            return 0
+        run_reference(args, pname, dname, peaks, peak_src, world)
+        return 0
+
+    import torch
+    import torch.distributed as dist
+
+    import flashattention_attention_attn_b200 as fa
+    from flashattention_attention_attn_b200 import build as _build, inputs, workloads
+
+    if not os.path.exists(_build.LIB_PATH):
+        _build.build()
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    if fa.attn_check_support(local_rank) != 0:
+        raise RuntimeError("device not supported by the library")
+
+    ps = inputs.WORKLOADS[pname]
+    ds = inputs.WORKLOADS[dname]
+    # weak scaling: every rank runs its own batch (different seeds), no exchange
+    q, k, v = inputs.make_prefill(ps, seed=ps.seed + 100 * rank)
+    dinp = inputs.make_paged(ds, seed=ds.seed + 100 * rank)
+    dq, dk, dv = q.to(dev), k.to(dev), v.to(dev)
+    o = torch.empty_like(dq)
+    lse = torch.empty(ps.B, ps.Hq, ps.T, device=dev, dtype=torch.float32)
+    qd_, kc, vc = dinp.q.to(dev), dinp.k_cache.to(dev), dinp.v_cache.to(dev)
+    bt, sl = dinp.block_table.to(dev), dinp.seq_lens.to(dev)
+    od = torch.empty(ds.B, ds.Hq, ds.d, device=dev, dtype=torch.bfloat16)
+    maxb = dinp.block_table.shape[1]
+    stream = torch.cuda.current_stream(dev)
+
+    flops = workloads.prefill_flops(ps.B, ps.Hq, ps.T, ps.S, ps.d, ps.causal)
+    dbytes = workloads.decode_bytes(dinp.seq_lens.tolist(), ds.Hq, ds.Hkv, ds.d, ds.block_size)
+    splits = args.num_splits
+
+    def step():
+        fa.attn_fwd(dq, dk, dv, o, lse, ps.B, ps.Hq, ps.Hkv, ps.T, ps.S, ps.d, ps.causal, ps.scale, stream)
+        fa.paged_attn_decode(qd_, kc, vc, bt, sl, ds.B, ds.Hq, ds.Hkv, ds.d, ds.block_size, maxb, splits, od,
+                             stream)
+
+    for _ in range(max(3, args.warmup)):
+        step()
+    torch.cuda.synchronize()
+
+    K = args.steps
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(K)]
+    start = torch.cuda.Event(enable_timing=True)
+    end = torch.cuda.Event(enable_timing=True)
+    sampler = ClockSampler(local_rank)
+    sampler.start()
+    time.sleep(0.05)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    t_wall0 = time.perf_counter()
+    start.record(stream)
+    for i in range(K):
+        ev[i][0].record(stream)
+        fa.attn_fwd(dq, dk, dv, o, lse, ps.B, ps.Hq, ps.Hkv, ps.T, ps.S, ps.d, ps.causal, ps.scale, stream)
+        ev[i][1].record(stream)
+        fa.paged_attn_decode(qd_, kc, vc, bt, sl, ds.B, ds.Hq, ds.Hkv, ds.d, ds.block_size, maxb, splits, od,
+                             stream)
+        ev[i][2].record(stream)
+    end.record(stream)
+    torch.cuda.synchronize()
+    t_wall1 = time.perf_counter()
+    if world > 1:
+        dist.barrier()
+    sampler.stop()
+    status = fa.attn_read_device_status(clear=True)
+    if status != 0:
+        raise RuntimeError(f"device status {status}: a bounded wait timed out")
+
+    total_ms = start.elapsed_time(end)
+    t_pre = sum(ev[i][0].elapsed_time(ev[i][1]) for i in range(K)) / K
+    t_dec = sum(ev[i][1].elapsed_time(ev[i][2]) for i in range(K)) / K
+    ms_step = total_ms / K
+    if world > 1:
+        t = torch.tensor([ms_step, t_pre, t_dec], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms_step, t_pre, t_dec = t.tolist()
+
+    ideal_pre = flops / (peaks["bf16_tflops"] * 1e12)
+    ideal_dec = dbytes / (peaks["hbm_gbs"] * 1e9)
+    ideal = ideal_pre + ideal_dec
+    value = 100.0 * world * ideal / (ms_step * 1e-3)
+
+    # ---------------- end to end through the public API, host buffers ----------------
+    e2e = None
+    if args.e2e_steps > 0:
+        pin = lambda t: t.pin_memory()  # noqa: E731
+        h_in = [pin(q), pin(k), pin(v), pin(dinp.q), pin(dinp.k_cache), pin(dinp.v_cache),
+                pin(dinp.block_table), pin(dinp.seq_lens)]
+        d_in = [dq, dk, dv, qd_, kc, vc, bt, sl]
+        h_o = torch.empty(o.shape, dtype=o.dtype).pin_memory()
+        h_lse = torch.empty(lse.shape, dtype=lse.dtype).pin_memory()
+        h_od = torch.empty(od.shape, dtype=od.dtype).pin_memory()
+        h2d = sum(t.numel() * t.element_size() for t in h_in)
+        d2h = sum(t.numel() * t.element_size() for t in (h_o, h_lse, h_od))
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+        e0.record(stream)
+        for _ in range(args.e2e_steps):
+            for h, d_ in zip(h_in, d_in):
+                d_.copy_(h, non_blocking=True)
+            step()
+            h_o.copy_(o, non_blocking=True)
+            h_lse.copy_(lse, non_blocking=True)
+            h_od.copy_(od, non_blocking=True)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        e2e_ms = e0.elapsed_time(e1) / args.e2e_steps
+        if world > 1:
+            t = torch.tensor([e2e_ms], device=dev)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            e2e_ms = t.item()
+        e2e = {"value": 100.0 * world * ideal / (e2e_ms * 1e-3), "unit": UNIT, "h2d_bytes_per_step": int(h2d),
+               "d2h_bytes_per_step": int(d2h), "ms_per_step": e2e_ms}
+
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank != 0:
+        return 0
+
+    dec_gbs = dbytes / (t_dec * 1e-3) / 1e9
+    pre_tflops = flops / (t_pre * 1e-3) / 1e12
+    dominant = "decode" if t_dec >= t_pre else "prefill"
+    if dominant == "decode":
+        roofline = {"bound": "hbm", "achieved": dec_gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                    "frac": dec_gbs / peaks["hbm_gbs"], "traffic": None,
+                    "kernel": "paged_attn_decode (split kernel + LSE combine)",
+                    "peak_source": f"{peak_src} (hbm_gbs)"}
+    else:
+        roofline = {"bound": "tensor", "achieved": pre_tflops, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                    "frac": pre_tflops / peaks["bf16_tflops"], "traffic": None, "kernel": "attn_fwd",
+                    "peak_source": f"{peak_src} (bf16_tflops, burst)"}
+    launches_per_step = 1 + 1 + 1  # prefill, decode split kernel, LSE combine
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K, "warmup": args.warmup,
+        "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16", "data": "synthetic (seeded N(0,1) bf16; random block-id permutations)",
+        "config": {"workload": f"{pname} + {dname}", "prefill": vars_of(ps), "decode": vars_of(ds),
+                   "decode_num_splits": splits or "auto", "parallelism": f"replicas x{world} (no exchange)",
+                   "l2": "inputs larger than L2 (decode KV cache %.0f MB per step)" % (dbytes / 1e6)},
+        "parts": {"prefill": {"ms": t_pre, "tflops": pre_tflops, "frac": pre_tflops / peaks["bf16_tflops"],
+                              "flops": flops},
+                  "decode": {"ms": t_dec, "gbs": dec_gbs, "frac": dec_gbs / peaks["hbm_gbs"],
+                             "bytes": dbytes}},
+        "roofline": roofline,
+        "e2e": e2e,
+        "gpu_launches": launches_per_step * K,
+        "clocks": sampler.summary(t_wall0, t_wall1),
+        "peaks": {**peaks, "source": peak_src},
+    }
+    if not args.no_cpu_baseline and world == 1:
+        cb = cpu_baseline(pname, dname, peaks)
+        cb.pop("est_step_s", None)
+        line["cpu_baseline"] = cb
+    print(json.dumps(line))
+    return 0
+
+
+def vars_of(spec):
+    return {k: getattr(spec, k) for k in spec.__dataclass_fields__ if not k.startswith("_")}
+
+
+def run_reference(args, pname, dname, peaks, peak_src, world):
+    """The fp64 CPU oracle, each step a bounded sample of the same workload."""
+    steps = []
+    info = None
+    for i in range(max(0, args.warmup) + args.steps):
+        budget = 20.0 / max(1, args.steps)
+        r = cpu_baseline(pname, dname, peaks, budget_s=budget)
+        if i >= args.warmup:
+            steps.append(r["est_step_s"])
+            info = r
+    est = sum(steps) / len(steps)
+    from flashattention_attention_attn_b200 import inputs
+    value = info["value"]
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": est * 1e3, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic (same seeds as ours)",
+        "config": {"workload": f"{pname} + {dname}", "prefill": vars_of(inputs.WORKLOADS[pname]),
+                   "decode": vars_of(inputs.WORKLOADS[dname])},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": info["cores"], "kind": "oracle",
+                         "sample": info["sample"]},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        "peaks": {**peaks, "source": peak_src},
+    }
+    print(json.dumps(line))
+
+
+if __name__ == "__main__":
+    sys.exit(main())

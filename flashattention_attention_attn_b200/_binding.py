@@ -1,0 +1,103 @@
+"""ctypes binding of the C ABI in include/attn.h.
+
+Argument marshalling only: tensors become device pointers, the current
+torch stream becomes the cudaStream_t, and a non-zero status becomes an
+exception.  Every step of the computation runs in the CUDA library; if it
+cannot be loaded, every call raises.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+library_path = os.path.join(os.path.dirname(os.path.abspath(__file__)), "_lib", "libattn_b200.so")
+
+ATTN_OK = 0
+_lib = None
+
+
+class AttnError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        self.status = status
+        super().__init__(f"{what}: {attn_status_string(status)} (status {status})")
+
+
+def library() -> ctypes.CDLL:
+    """Load the library once (raises if it is missing: there is no fallback)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(library_path):
+            raise RuntimeError(
+                f"CUDA library not built: {library_path} is missing "
+                "(run `python -m flashattention_attention_attn_b200.build`)")
+        lib = ctypes.CDLL(library_path)
+        c_int, c_float, vp = ctypes.c_int, ctypes.c_float, ctypes.c_void_p
+        lib.attn_fwd.argtypes = [vp, vp, vp, vp, vp, c_int, c_int, c_int, c_int, c_int, c_int, c_int, c_float, vp]
+        lib.attn_fwd.restype = c_int
+        lib.paged_attn_decode.argtypes = [vp, vp, vp, vp, vp, c_int, c_int, c_int, c_int, c_int, c_int, c_int,
+                                          vp, vp]
+        lib.paged_attn_decode.restype = c_int
+        lib.attn_check_support.argtypes = [c_int]
+        lib.attn_check_support.restype = c_int
+        lib.attn_status_string.argtypes = [c_int]
+        lib.attn_status_string.restype = ctypes.c_char_p
+        lib.attn_read_device_status.argtypes = [ctypes.POINTER(c_int), c_int]
+        lib.attn_read_device_status.restype = c_int
+        _lib = lib
+    return _lib
+
+
+def _ptr(x) -> int | None:
+    if x is None:
+        return None
+    if isinstance(x, torch.Tensor):
+        return x.data_ptr() if x.numel() > 0 else None
+    return int(x)
+
+
+def _stream(stream) -> int | None:
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, torch.cuda.Stream):
+        return stream.cuda_stream
+    return int(stream)
+
+
+def attn_status_string(status: int) -> str:
+    return library().attn_status_string(int(status)).decode()
+
+
+def attn_fwd(q, k, v, o, lse, B, Hq, Hkv, T, S, d, causal, scale, stream=None) -> None:
+    """O = softmax(scale * Q K^T [+ causal mask]) V, plus LSE.
+
+    q [B,T,Hq,d], k/v [B,S,Hkv,d], o [B,T,Hq,d] bf16; lse [B,Hq,T] fp32 or None.
+    """
+    rc = library().attn_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), int(B), int(Hq), int(Hkv), int(T),
+                            int(S), int(d), int(bool(causal)), float(scale), _stream(stream))
+    if rc != ATTN_OK:
+        raise AttnError(rc, "attn_fwd")
+
+
+def paged_attn_decode(q, k_cache, v_cache, block_table, seq_lens, B, Hq, Hkv, d, block_size, max_blocks,
+                      num_splits, o, stream=None) -> None:
+    """One query token per sequence against a paged KV cache (see attn.h)."""
+    rc = library().paged_attn_decode(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_table), _ptr(seq_lens),
+                                     int(B), int(Hq), int(Hkv), int(d), int(block_size), int(max_blocks),
+                                     int(num_splits), _ptr(o), _stream(stream))
+    if rc != ATTN_OK:
+        raise AttnError(rc, "paged_attn_decode")
+
+
+def attn_check_support(device: int = 0) -> int:
+    return int(library().attn_check_support(int(device)))
+
+
+def attn_read_device_status(clear: bool = True) -> int:
+    out = ctypes.c_int(0)
+    rc = library().attn_read_device_status(ctypes.byref(out), int(bool(clear)))
+    if rc != ATTN_OK:
+        raise AttnError(rc, "attn_read_device_status")
+    return int(out.value)

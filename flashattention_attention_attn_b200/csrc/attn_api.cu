@@ -1,0 +1,350 @@
+// attn_api.cu - host side of the C ABI declared in include/attn.h: argument
+// validation, TMA descriptor construction, launch configuration and the
+// stream-ordered workspace of the split-KV decode.  Every step of the
+// computation runs in the kernels included below; there is no CPU path.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "attn.h"
+#include "decode_paged.cuh"
+#include "prefill_sm100.cuh"
+#include "sm100_ptx.cuh"
+
+namespace attn {
+namespace {
+
+constexpr int kMaxDevices = 64;
+
+__global__ void fill_no_keys(__nv_bfloat16* o, float* lse, size_t n_o, size_t n_lse) {
+  const size_t i = static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  const size_t stride = static_cast<size_t>(gridDim.x) * blockDim.x;
+  for (size_t k = i; k < n_o; k += stride) o[k] = __float2bfloat16_rn(0.f);
+  if (lse != nullptr)
+    for (size_t k = i; k < n_lse; k += stride) lse[k] = -INFINITY;
+}
+
+struct DeviceState {
+  bool probed = false;
+  int status = ATTN_ERR_CUDA;  // result of the support check
+  int sms = 0;
+  bool attrs_set = false;
+  cudaMemPool_t pool = nullptr;
+};
+
+std::mutex g_mu;
+DeviceState g_dev[kMaxDevices];
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_tiled() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+  });
+  return fn;
+}
+
+// Probe a device once: sm_100 (compute capability 10.0) and a loadable image.
+int probe_device(int dev, DeviceState** out) {
+  if (dev < 0 || dev >= kMaxDevices) return ATTN_ERR_INVALID_ARG;
+  std::lock_guard<std::mutex> lock(g_mu);
+  DeviceState& st = g_dev[dev];
+  if (!st.probed) {
+    int major = 0, minor = 0, sms = 0;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) {
+      cudaGetLastError();
+      st.status = ATTN_ERR_CUDA;
+    } else if (major != 10 || minor != 0) {
+      st.status = ATTN_ERR_UNSUPPORTED;
+    } else {
+      cudaFuncAttributes fa;
+      if (cudaFuncGetAttributes(&fa, prefill::prefill_fwd_sm100<128>) != cudaSuccess) {
+        cudaGetLastError();
+        st.status = ATTN_ERR_UNSUPPORTED;  // no sm_100a image for this device
+      } else if (encode_tiled() == nullptr) {
+        st.status = ATTN_ERR_CUDA;
+      } else {
+        st.status = ATTN_OK;
+      }
+    }
+    st.sms = sms;
+    st.probed = true;
+  }
+  *out = &st;
+  return st.status;
+}
+
+// Per-device one-time launch set-up (dynamic shared memory limits, pool).
+int prepare_device(int dev, DeviceState* st) {
+  std::lock_guard<std::mutex> lock(g_mu);
+  if (st->attrs_set) return ATTN_OK;
+  const struct {
+    const void* fn;
+    size_t bytes;
+  } kernels[] = {
+      {reinterpret_cast<const void*>(prefill::prefill_fwd_sm100<64>), prefill::smem_bytes<64>()},
+      {reinterpret_cast<const void*>(prefill::prefill_fwd_sm100<128>), prefill::smem_bytes<128>()},
+      {reinterpret_cast<const void*>(decode::paged_decode_split<64>), decode::smem_bytes<64>()},
+      {reinterpret_cast<const void*>(decode::paged_decode_split<128>), decode::smem_bytes<128>()},
+  };
+  for (const auto& k : kernels)
+    if (cudaFuncSetAttribute(k.fn, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(k.bytes)) !=
+        cudaSuccess) {
+      cudaGetLastError();
+      return ATTN_ERR_CUDA;
+    }
+  cudaMemPoolProps props;
+  std::memset(&props, 0, sizeof(props));
+  props.allocType = cudaMemAllocationTypePinned;
+  props.location.type = cudaMemLocationTypeDevice;
+  props.location.id = dev;
+  if (cudaMemPoolCreate(&st->pool, &props) != cudaSuccess) {
+    cudaGetLastError();
+    return ATTN_ERR_CUDA;
+  }
+  uint64_t keep = UINT64_MAX;  // keep freed workspace cached in the pool
+  cudaMemPoolSetAttribute(st->pool, cudaMemPoolAttrReleaseThreshold, &keep);
+  st->attrs_set = true;
+  return ATTN_OK;
+}
+
+int current_device_state(DeviceState** st) {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess) {
+    cudaGetLastError();
+    return ATTN_ERR_CUDA;
+  }
+  int rc = probe_device(dev, st);
+  if (rc != ATTN_OK) return rc;
+  return prepare_device(dev, *st);
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// 4-D bf16 map over a [B, rows, H, D] tensor: dims (D, H, rows, B),
+// box (64, 1, 128, 1), 128-byte swizzle.
+int make_map_bthd(CUtensorMap* map, const void* base, int B, int rows, int H, int D) {
+  cuuint64_t dims[4] = {cuuint64_t(D), cuuint64_t(H), cuuint64_t(rows), cuuint64_t(B)};
+  cuuint64_t strides[3] = {cuuint64_t(D) * 2, cuuint64_t(H) * D * 2, cuuint64_t(rows) * H * D * 2};
+  cuuint32_t box[4] = {64, 1, 128, 1};
+  cuuint32_t estr[4] = {1, 1, 1, 1};
+  CUresult r = encode_tiled()(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides,
+                              box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? ATTN_OK : ATTN_ERR_CUDA;
+}
+
+// 2-D bf16 map over a paged pool seen as [tokens, Hkv * D]: box (64, 16).
+// The pool size is not part of the call, so the token extent is the largest
+// the coordinates can address; only block ids read from the table are used.
+int make_map_pool(CUtensorMap* map, const void* base, int Hkv, int D) {
+  constexpr cuuint64_t kTokens = (1ull << 31) - 16;
+  cuuint64_t dims[2] = {cuuint64_t(Hkv) * D, kTokens};
+  cuuint64_t strides[1] = {cuuint64_t(Hkv) * D * 2};
+  cuuint32_t box[2] = {64, 16};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = encode_tiled()(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides,
+                              box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? ATTN_OK : ATTN_ERR_CUDA;
+}
+
+int launch_status() {
+  cudaError_t e = cudaGetLastError();
+  return e == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+}
+
+template <int D>
+int launch_prefill(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq, int Hkv,
+                   int T, int S, int causal, float scale, cudaStream_t stream) {
+  CUtensorMap mq, mk, mv, mo;
+  if (make_map_bthd(&mq, q, B, T, Hq, D) || make_map_bthd(&mk, k, B, S, Hkv, D) ||
+      make_map_bthd(&mv, v, B, S, Hkv, D) || make_map_bthd(&mo, o, B, T, Hq, D))
+    return ATTN_ERR_CUDA;
+  prefill::Params p;
+  p.lse = lse;
+  p.B = B;
+  p.Hq = Hq;
+  p.Hkv = Hkv;
+  p.T = T;
+  p.S = S;
+  p.causal = causal ? 1 : 0;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  p.num_mblocks = (T + 2 * prefill::kBM - 1) / (2 * prefill::kBM);
+  const long long grid = static_cast<long long>(p.num_mblocks) * Hq * B;
+  if (grid > 0x7fffffffLL) return ATTN_ERR_UNSUPPORTED;
+  prefill::prefill_fwd_sm100<D><<<static_cast<unsigned>(grid), prefill::kThreads, prefill::smem_bytes<D>(),
+                                  stream>>>(mq, mk, mv, mo, p);
+  return launch_status();
+}
+
+// Splits chosen so that the CTAs of a batch whose sequences all reach
+// max_blocks fill the GPU about twice (2 CTAs of the decode kernel fit on
+// one SM), with at least 8 blocks per split.
+int auto_splits(int B, int groups, int max_blocks, int sms) {
+  const long long units = static_cast<long long>(B) * groups;
+  const long long target = 4LL * sms;
+  long long splits = (target + units - 1) / units;
+  const long long max_splits = (max_blocks + 7) / 8;
+  if (splits > max_splits) splits = max_splits;
+  if (splits < 1) splits = 1;
+  return static_cast<int>(splits);
+}
+
+template <int D>
+int launch_decode(const void* q, const void* kc, const void* vc, const int32_t* table, const int32_t* lens, int B,
+                  int Hq, int Hkv, int max_blocks, int num_splits, void* o, cudaStream_t stream,
+                  const DeviceState* st) {
+  CUtensorMap mk, mv;
+  if (make_map_pool(&mk, kc, Hkv, D) || make_map_pool(&mv, vc, Hkv, D)) return ATTN_ERR_CUDA;
+  const int groups = (Hkv + decode::kKH - 1) / decode::kKH;
+  if (num_splits <= 0) num_splits = auto_splits(B, groups, max_blocks, st->sms);
+  if (num_splits > max_blocks) num_splits = max_blocks;
+  const int chunk = (max_blocks + num_splits - 1) / num_splits;
+  num_splits = (max_blocks + chunk - 1) / chunk;  // drop splits that can never hold a block
+  if (num_splits > 65535 || groups > 65535 || B > 65535) return ATTN_ERR_UNSUPPORTED;
+
+  decode::Params p;
+  p.q = static_cast<const __nv_bfloat16*>(q);
+  p.block_table = table;
+  p.seq_lens = lens;
+  p.o = static_cast<__nv_bfloat16*>(o);
+  p.part_o = nullptr;
+  p.part_lse = nullptr;
+  p.B = B;
+  p.Hq = Hq;
+  p.Hkv = Hkv;
+  p.max_blocks = max_blocks;
+  p.num_splits = num_splits;
+  p.chunk = chunk;
+  p.scale_log2 = (1.0f / std::sqrt(static_cast<float>(D))) * 1.4426950408889634f;
+
+  void* ws = nullptr;
+  if (num_splits > 1) {
+    const size_t rows = static_cast<size_t>(num_splits) * B * Hq;
+    const size_t bytes = rows * D * sizeof(float) + rows * sizeof(float);
+    if (cudaMallocFromPoolAsync(&ws, bytes, st->pool, stream) != cudaSuccess) {
+      cudaGetLastError();
+      return ATTN_ERR_CUDA;
+    }
+    p.part_o = static_cast<float*>(ws);
+    p.part_lse = p.part_o + rows * D;
+  }
+  dim3 grid(num_splits, groups, B);
+  decode::paged_decode_split<D><<<grid, (decode::kKH + 1) * 32, decode::smem_bytes<D>(), stream>>>(mk, mv, p);
+  int rc = launch_status();
+  if (rc == ATTN_OK && num_splits > 1) {
+    dim3 cgrid(Hq, B, D / 32);
+    decode::lse_combine<D><<<cgrid, 128, 0, stream>>>(p.part_o, p.part_lse, lens, p.o, B, Hq, num_splits, chunk);
+    rc = launch_status();
+  }
+  if (ws != nullptr) cudaFreeAsync(ws, stream);
+  return rc;
+}
+
+}  // namespace
+}  // namespace attn
+
+using namespace attn;
+
+extern "C" int attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq, int Hkv,
+                        int T, int S, int d, int causal, float scale, attn_stream_t stream_) {
+  cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+  if (B < 0 || T < 0 || S < 0 || Hq <= 0 || Hkv <= 0 || d <= 0) return ATTN_ERR_INVALID_ARG;
+  if (Hq % Hkv != 0) return ATTN_ERR_INVALID_ARG;
+  if (!(scale > 0.f) || !std::isfinite(scale)) return ATTN_ERR_INVALID_ARG;
+  if (B == 0 || T == 0) return ATTN_OK;
+  if (q == nullptr || o == nullptr || (S > 0 && (k == nullptr || v == nullptr))) return ATTN_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return ATTN_ERR_UNSUPPORTED;
+  if (!aligned16(q) || !aligned16(o) || (S > 0 && (!aligned16(k) || !aligned16(v)))) return ATTN_ERR_UNSUPPORTED;
+  if (lse != nullptr && (reinterpret_cast<uintptr_t>(lse) & 3u)) return ATTN_ERR_UNSUPPORTED;
+  DeviceState* st = nullptr;
+  int rc = current_device_state(&st);
+  if (rc != ATTN_OK) return rc;
+  if (S == 0) {  // no key at all: O = 0, LSE = -inf
+    const size_t n_o = static_cast<size_t>(B) * T * Hq * d;
+    const size_t n_lse = static_cast<size_t>(B) * Hq * T;
+    fill_no_keys<<<st->sms * 4, 256, 0, stream>>>(static_cast<__nv_bfloat16*>(o), lse, n_o, n_lse);
+    return launch_status();
+  }
+  if (d == 64) return launch_prefill<64>(q, k, v, o, lse, B, Hq, Hkv, T, S, causal, scale, stream);
+  return launch_prefill<128>(q, k, v, o, lse, B, Hq, Hkv, T, S, causal, scale, stream);
+}
+
+extern "C" int paged_attn_decode(const void* q, const void* k_cache, const void* v_cache,
+                                 const int32_t* block_table, const int32_t* seq_lens, int B, int Hq, int Hkv, int d,
+                                 int block_size, int max_blocks, int num_splits, void* o, attn_stream_t stream_) {
+  cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+  if (B < 0 || Hq <= 0 || Hkv <= 0 || d <= 0 || block_size <= 0) return ATTN_ERR_INVALID_ARG;
+  if (Hq % Hkv != 0) return ATTN_ERR_INVALID_ARG;
+  if (B == 0) return ATTN_OK;
+  if (max_blocks <= 0) return ATTN_ERR_INVALID_ARG;
+  if (q == nullptr || k_cache == nullptr || v_cache == nullptr || block_table == nullptr || seq_lens == nullptr ||
+      o == nullptr)
+    return ATTN_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return ATTN_ERR_UNSUPPORTED;
+  if (block_size != decode::kBlock) return ATTN_ERR_UNSUPPORTED;
+  if (Hq / Hkv > 8) return ATTN_ERR_UNSUPPORTED;
+  if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(o)) return ATTN_ERR_UNSUPPORTED;
+  if ((reinterpret_cast<uintptr_t>(block_table) & 3u) || (reinterpret_cast<uintptr_t>(seq_lens) & 3u))
+    return ATTN_ERR_UNSUPPORTED;
+  DeviceState* st = nullptr;
+  int rc = current_device_state(&st);
+  if (rc != ATTN_OK) return rc;
+  if (d == 64)
+    return launch_decode<64>(q, k_cache, v_cache, block_table, seq_lens, B, Hq, Hkv, max_blocks, num_splits, o,
+                             stream, st);
+  return launch_decode<128>(q, k_cache, v_cache, block_table, seq_lens, B, Hq, Hkv, max_blocks, num_splits, o,
+                            stream, st);
+}
+
+extern "C" int attn_check_support(int device) {
+  DeviceState* st = nullptr;
+  return probe_device(device, &st);
+}
+
+extern "C" const char* attn_status_string(int status) {
+  switch (status) {
+    case ATTN_OK:
+      return "ok";
+    case ATTN_ERR_INVALID_ARG:
+      return "invalid argument";
+    case ATTN_ERR_UNSUPPORTED:
+      return "unsupported (shape, alignment or device)";
+    case ATTN_ERR_CUDA:
+      return "CUDA error";
+    case ATTN_ERR_TIMEOUT:
+      return "device-side wait timed out";
+    default:
+      return "unknown status";
+  }
+}
+
+extern "C" int attn_read_device_status(int* out, int clear) {
+  if (out == nullptr) return ATTN_ERR_INVALID_ARG;
+  int v = 0;
+  if (cudaMemcpyFromSymbol(&v, attn::g_devstatus, sizeof(int)) != cudaSuccess) {
+    cudaGetLastError();
+    return ATTN_ERR_CUDA;
+  }
+  *out = v;
+  if (clear && v != 0) {
+    const int zero = 0;
+    if (cudaMemcpyToSymbol(attn::g_devstatus, &zero, sizeof(int)) != cudaSuccess) {
+      cudaGetLastError();
+      return ATTN_ERR_CUDA;
+    }
+  }
+  return ATTN_OK;
+}

@@ -1,0 +1,378 @@
+// prefill_sm100.cuh - fused causal / non-causal GQA attention forward for
+// sm_100a: TMA tile loads, tcgen05 MMAs with accumulators in tensor memory,
+// online softmax in registers, warp-specialised roles.
+//
+// What it computes is the blockwise scheme of the page "Snelle
+// attention-kernels en operatorfusie versnellen AI-modellen" (the-ai.news),
+// section "FlashAttention-type aandacht en gepagineerde aandacht": for each
+// key/value block, form that block's scores, update the running softmax
+// statistics (row max, row sum) and accumulate the output on chip; the full
+// score matrix is never written out.
+//
+// CTA = two 128-row query tiles (rows m0..m0+255) of one (batch, q-head).
+//   warps 0-3  softmax for query tile 0 (thread r owns row r = TMEM lane r)
+//   warps 4-7  softmax for query tile 1
+//   warp  8    TMA producer (Q once, then a K ring and a V ring)
+//   warp  9    MMA issuer (one thread): S_t = Q_t K^T, O_t += P_t V
+// Tensor memory (512 columns x 128 lanes x 32 bit):
+//   S_0 cols [0,128), S_1 [128,256): fp32 scores; after the softmax the same
+//   columns hold P as packed bf16 (64 columns), the A operand of P V.
+//   O_0 [256, 256+D), O_1 [256+D, 256+2D): fp32 output accumulators.
+// The two query tiles ping-pong: while the softmax warps of one tile work,
+// the tensor core runs the other tile's MMAs.
+//
+// Softmax statistics are kept in the log2 domain (s * scale * log2 e) and the
+// exponentials use ex2.  The row max used as reference is only moved (and O
+// rescaled by exp2(m_old - m_new)) when the new max exceeds it by more than
+// kRescaleThreshold; otherwise P carries values up to 2^threshold, which fp32
+// accumulation and bf16 P (same exponent range as fp32) absorb.  O and the row
+// sum always share the same reference, so the final O / l is unchanged.
+#pragma once
+
+#include "sm100_ptx.cuh"
+
+namespace attn {
+namespace prefill {
+
+constexpr int kBM = 128;               // rows per query tile (= TMEM lanes)
+constexpr int kBN = 128;               // keys per K/V tile
+constexpr int kThreads = 320;          // 10 warps
+constexpr int kWarpLoad = 8;
+constexpr int kWarpMma = 9;
+constexpr float kRescaleThreshold = 8.0f;  // log2 units
+constexpr uint32_t kTmemCols = 512;
+
+template <int D>
+struct Config {
+  static constexpr int kChunks = D / 64;                     // 128-byte swizzle chunks per row
+  static constexpr int kStages = (D == 64) ? 4 : 2;          // K ring depth = V ring depth
+  static constexpr uint32_t kTileBytes = kBM * D * 2;        // one Q / K / V tile (bf16)
+  static constexpr uint32_t kChunkBytes = kBM * 128;         // 128 rows x 128 bytes
+};
+
+template <int D>
+struct __align__(1024) Smem {
+  using C = Config<D>;
+  __nv_bfloat16 q[2][C::kChunks][kBM * 64];
+  __nv_bfloat16 k[C::kStages][C::kChunks][kBN * 64];
+  __nv_bfloat16 v[C::kStages][C::kChunks][kBN * 64];
+  uint64_t q_full[2];
+  uint64_t k_full[C::kStages], k_empty[C::kStages];
+  uint64_t v_full[C::kStages], v_empty[C::kStages];
+  uint64_t s_full[2], p_full[2], o_full[2];
+  uint64_t mma_done;
+  uint32_t tmem_base;
+  int abort_flag;
+};
+
+template <int D>
+constexpr size_t smem_bytes() {
+  return sizeof(Smem<D>) + 1024;  // + slack to align the dynamic base to 1024
+}
+
+struct Params {
+  float* lse;  // [B, Hq, T] or nullptr
+  int B, Hq, Hkv, T, S;
+  int causal;
+  float scale_log2;  // scale * log2(e)
+  int num_mblocks;   // ceil(T / 256)
+};
+
+// Keys visible to the query tile with rows [r0, r0 + 128) (ragged T clipped)
+// as a number of kBN-wide K/V tiles; 0 when no row of it sees any key.
+__device__ __forceinline__ int kv_tiles_for(int r0, const Params& p) {
+  if (r0 >= p.T) return 0;
+  const int r1 = min(r0 + kBM, p.T);
+  int kmax = p.S - 1;
+  if (p.causal) kmax = min(kmax, r1 - 1 + (p.S - p.T));
+  if (kmax < 0) return 0;
+  return kmax / kBN + 1;
+}
+
+template <int D>
+__global__ void __launch_bounds__(kThreads, 1)
+    prefill_fwd_sm100(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                      const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
+                      const Params p) {
+  using C = Config<D>;
+  extern __shared__ uint8_t smem_raw[];
+  Smem<D>& sm = *reinterpret_cast<Smem<D>*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  // Work tile: heaviest (last) query blocks first; adjacent CTAs are adjacent
+  // q heads of one (block, batch) so the heads sharing a KV head run together.
+  const int per_mb = p.Hq * p.B;
+  const int mb = p.num_mblocks - 1 - static_cast<int>(blockIdx.x) / per_mb;
+  const int rem = static_cast<int>(blockIdx.x) % per_mb;
+  const int h = rem % p.Hq;
+  const int b = rem / p.Hq;
+  const int hk = h / (p.Hq / p.Hkv);
+  const int m0 = mb * 2 * kBM;
+  const int n0 = kv_tiles_for(m0, p);
+  const int n1 = kv_tiles_for(m0 + kBM, p);
+  const int n_max = max(n0, n1);
+
+  if (threadIdx.x == 0) {
+    for (int t = 0; t < 2; ++t) {
+      mbar_init(&sm.q_full[t], 1);
+      mbar_init(&sm.s_full[t], 1);
+      mbar_init(&sm.p_full[t], kBM);
+      mbar_init(&sm.o_full[t], 1);
+    }
+    for (int s = 0; s < C::kStages; ++s) {
+      mbar_init(&sm.k_full[s], 1);
+      mbar_init(&sm.k_empty[s], 1);
+      mbar_init(&sm.v_full[s], 1);
+      mbar_init(&sm.v_empty[s], 1);
+    }
+    mbar_init(&sm.mma_done, 1);
+    sm.abort_flag = 0;
+    fence_mbarrier_init();
+  }
+  if (warp == 0) {
+    tmem_alloc(&sm.tmem_base, kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = sm.tmem_base;
+  volatile int* abort_flag = &sm.abort_flag;
+
+  if (warp == kWarpLoad) {
+    // ------------------------------ producer ------------------------------
+    if (lane == 0) {
+      tma_prefetch_desc(&tmQ);
+      tma_prefetch_desc(&tmK);
+      tma_prefetch_desc(&tmV);
+      const int nt[2] = {n0, n1};
+      for (int t = 0; t < 2; ++t) {
+        if (nt[t] == 0) continue;
+        mbar_arrive_expect_tx(&sm.q_full[t], C::kTileBytes);
+        for (int c = 0; c < C::kChunks; ++c)
+          tma_load_4d(sm.q[t][c], &tmQ, &sm.q_full[t], c * 64, h, m0 + t * kBM, b);
+      }
+      int k_issued = 0, v_issued = 0;  // K / V tiles whose loads were issued
+      for (int j = 0; j < n_max; ++j) {
+        const int s = j % C::kStages;
+        const uint32_t ph = (j / C::kStages) & 1;
+        if (!mbar_wait(&sm.k_empty[s], ph ^ 1, abort_flag)) break;
+        mbar_arrive_expect_tx(&sm.k_full[s], C::kTileBytes);
+        for (int c = 0; c < C::kChunks; ++c)
+          tma_load_4d(sm.k[s][c], &tmK, &sm.k_full[s], c * 64, hk, j * kBN, b);
+        k_issued = j + 1;
+        if (!mbar_wait(&sm.v_empty[s], ph ^ 1, abort_flag)) break;
+        mbar_arrive_expect_tx(&sm.v_full[s], C::kTileBytes);
+        for (int c = 0; c < C::kChunks; ++c)
+          tma_load_4d(sm.v[s][c], &tmV, &sm.v_full[s], c * 64, hk, j * kBN, b);
+        v_issued = j + 1;
+      }
+      if (*abort_flag) {
+        // Let the copies already issued land before shared memory is released.
+        for (int t = 0; t < 2; ++t)
+          if (nt[t] > 0) mbar_wait_drain(&sm.q_full[t], 0);
+        for (int j = max(0, k_issued - C::kStages); j < k_issued; ++j)
+          mbar_wait_drain(&sm.k_full[j % C::kStages], (j / C::kStages) & 1);
+        for (int j = max(0, v_issued - C::kStages); j < v_issued; ++j)
+          mbar_wait_drain(&sm.v_full[j % C::kStages], (j / C::kStages) & 1);
+      }
+    }
+  } else if (warp == kWarpMma) {
+    // ---------------------------- MMA issuer ------------------------------
+    if (lane == 0) {
+      constexpr uint32_t idesc_qk = make_idesc_bf16(kBM, kBN, 0, 0);  // Q, K both K-major
+      constexpr uint32_t idesc_pv = make_idesc_bf16(kBM, D, 0, 1);    // P (TMEM), V MN-major
+      const int nt[2] = {n0, n1};
+      bool ok = true;
+      for (int t = 0; t < 2 && ok; ++t)
+        if (nt[t] > 0) ok = mbar_wait(&sm.q_full[t], 0, abort_flag);
+
+      // O_t += P_t(jj) V(jj)
+      auto issue_pv = [&](int t, int jj) -> bool {
+        const int s = jj % C::kStages;
+        if (!mbar_wait(&sm.v_full[s], (jj / C::kStages) & 1, abort_flag)) return false;
+        if (!mbar_wait(&sm.p_full[t], jj & 1, abort_flag)) return false;
+        tc_fence_after();
+        const uint32_t tS = tmem + t * kBN;
+        const uint32_t tO = tmem + 2 * kBN + t * D;
+        const uint32_t vbase = smem_u32(sm.v[s][0]);
+#pragma unroll
+        for (int kk = 0; kk < kBN / 16; ++kk) {
+          // 16 keys per step: 16 rows x 128 B further into each V chunk;
+          // LBO = distance between 64-wide d chunks, SBO = 8 rows x 128 B.
+          const uint64_t bdesc = make_sdesc_sw128(vbase + kk * 16 * 128, C::kChunkBytes, 1024);
+          umma_ts(tO, tS + kk * 8, bdesc, idesc_pv, (jj > 0 || kk > 0) ? 1u : 0u);
+        }
+        umma_commit(&sm.o_full[t]);
+        return true;
+      };
+
+      for (int j = 0; j < n_max && ok; ++j) {
+        const int s = j % C::kStages;
+        if (!(ok = mbar_wait(&sm.k_full[s], (j / C::kStages) & 1, abort_flag))) break;
+        tc_fence_after();
+        for (int t = 0; t < 2 && ok; ++t) {
+          // the previous P_t must be consumed before S_t is overwritten
+          if (j >= 1 && j - 1 < nt[t]) ok = issue_pv(t, j - 1);
+          if (ok && j < nt[t]) {
+            const uint32_t tS = tmem + t * kBN;
+            const uint32_t qbase = smem_u32(sm.q[t][0]);
+            const uint32_t kbase = smem_u32(sm.k[s][0]);
+#pragma unroll
+            for (int kk = 0; kk < D / 16; ++kk) {
+              const uint32_t off = (kk / 4) * C::kChunkBytes + (kk % 4) * 32;
+              const uint64_t adesc = make_sdesc_sw128(qbase + off, 16, 1024);
+              const uint64_t bdesc = make_sdesc_sw128(kbase + off, 16, 1024);
+              umma_ss(tS, adesc, bdesc, idesc_qk, kk > 0 ? 1u : 0u);
+            }
+            umma_commit(&sm.s_full[t]);
+          }
+        }
+        if (!ok) break;
+        umma_commit(&sm.k_empty[s]);
+        if (j >= 1) umma_commit(&sm.v_empty[(j - 1) % C::kStages]);
+      }
+      if (ok && n_max > 0) {
+        const int jl = n_max - 1;
+        for (int t = 0; t < 2 && ok; ++t)
+          if (jl < nt[t]) ok = issue_pv(t, jl);
+        if (ok) umma_commit(&sm.v_empty[jl % C::kStages]);
+      }
+      // Every MMA issued above is complete once mma_done fires; after an
+      // abort this keeps tensor memory allocated until they have finished.
+      umma_commit(&sm.mma_done);
+      mbar_wait_drain(&sm.mma_done, 0);
+    }
+  } else {
+    // ------------------------------ softmax -------------------------------
+    const int t = warp >> 2;              // query tile of this warpgroup
+    const int r = threadIdx.x & 127;      // row within the tile = TMEM lane
+    const int row = m0 + t * kBM + r;
+    const int nt = t ? n1 : n0;
+    const uint32_t lane_off = uint32_t((warp & 3) * 32) << 16;
+    const uint32_t tS = tmem + lane_off + t * kBN;
+    const uint32_t tO = tmem + lane_off + 2 * kBN + t * D;
+    const int visible = p.causal ? min(p.S, row + (p.S - p.T) + 1) : p.S;
+    const float sl2 = p.scale_log2;
+
+    float m_used = -INFINITY;  // reference max, log2 domain
+    float l = 0.f;             // running row sum relative to m_used
+    bool ok = true;
+    for (int j = 0; j < nt; ++j) {
+      ok = __all_sync(0xffffffffu, mbar_wait(&sm.s_full[t], j & 1, abort_flag));
+      if (!ok) break;
+      tc_fence_after();
+      float s[kBN];
+      {
+        uint32_t u[kBN];
+        tmem_ld128_sync(tS, u);
+#pragma unroll
+        for (int i = 0; i < kBN; ++i) s[i] = __uint_as_float(u[i]);
+      }
+      const int lim = visible - j * kBN;  // visible columns of this tile
+      if (lim < kBN) {
+#pragma unroll
+        for (int i = 0; i < kBN; ++i)
+          if (i >= lim) s[i] = -INFINITY;
+      }
+      float mx8[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) mx8[i] = s[i];
+#pragma unroll
+      for (int i = 8; i < kBN; ++i) mx8[i & 7] = fmaxf(mx8[i & 7], s[i]);
+      float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
+                       fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
+      const float m_new = fmaxf(m_used, mx * sl2);
+      if (m_new - m_used > kRescaleThreshold) {  // false while both are -inf (NaN)
+        if (m_used != -INFINITY) {
+          // O_t already holds P V of earlier tiles (their MMAs completed
+          // before this tile's S was committed): rescale it in place.
+          const float alpha = ex2_approx(m_used - m_new);
+          l *= alpha;
+#pragma unroll
+          for (int c = 0; c < D / 32; ++c) {
+            uint32_t u[32];
+            tmem_ld32_sync(tO + c * 32, u);
+#pragma unroll
+            for (int i = 0; i < 32; ++i) u[i] = __float_as_uint(__uint_as_float(u[i]) * alpha);
+            tmem_st_x32(tO + c * 32, u);
+          }
+        }
+        m_used = m_new;
+      }
+      const float mref = (m_used == -INFINITY) ? 0.f : m_used;
+      float sum8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+      for (int c = 0; c < kBN / 32; ++c) {
+        uint32_t pk[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          const float p0 = ex2_approx(fmaf(s[c * 32 + 2 * i], sl2, -mref));
+          const float p1 = ex2_approx(fmaf(s[c * 32 + 2 * i + 1], sl2, -mref));
+          sum8[(2 * i) & 7] += p0;
+          sum8[(2 * i + 1) & 7] += p1;
+          pk[i] = pack_bf16x2(p0, p1);
+        }
+        tmem_st_x16(tS + c * 16, pk);  // P overwrites the first 64 columns of S
+      }
+      l += ((sum8[0] + sum8[1]) + (sum8[2] + sum8[3])) + ((sum8[4] + sum8[5]) + (sum8[6] + sum8[7]));
+      tmem_st_wait();
+      tc_fence_before();
+      mbar_arrive(&sm.p_full[t]);
+    }
+
+    if (ok && nt > 0) {
+      ok = __all_sync(0xffffffffu, mbar_wait(&sm.o_full[t], (nt - 1) & 1, abort_flag));
+      tc_fence_after();
+    }
+    // Epilogue: O / l -> bf16, staged (128-byte swizzled) in this tile's Q
+    // buffer, then one TMA store per 64-wide chunk (rows >= T are clipped).
+    const float inv_l = (l > 0.f) ? 1.0f / l : 0.f;
+    const bool have_o = ok && nt > 0;
+    uint8_t* stage = reinterpret_cast<uint8_t*>(sm.q[t][0]);
+#pragma unroll
+    for (int c = 0; c < D / 32; ++c) {
+      uint32_t u[32];
+      if (have_o) {
+        tmem_ld32_sync(tO + c * 32, u);
+      } else {
+#pragma unroll
+        for (int i = 0; i < 32; ++i) u[i] = 0u;
+      }
+      uint32_t pk[16];
+#pragma unroll
+      for (int i = 0; i < 16; ++i)
+        pk[i] = pack_bf16x2(__uint_as_float(u[2 * i]) * inv_l, __uint_as_float(u[2 * i + 1]) * inv_l);
+      uint8_t* chunk = stage + (c / 2) * C::kChunkBytes + r * 128;
+#pragma unroll
+      for (int q4 = 0; q4 < 4; ++q4) {
+        const int unit = (c & 1) * 4 + q4;  // 16-byte unit within the 128-byte row
+        *reinterpret_cast<uint4*>(chunk + ((unit ^ (r & 7)) << 4)) =
+            make_uint4(pk[4 * q4], pk[4 * q4 + 1], pk[4 * q4 + 2], pk[4 * q4 + 3]);
+      }
+    }
+    if (p.lse != nullptr && row < p.T) {
+      const float lse = (l > 0.f) ? (m_used + __log2f(l)) * 0.69314718055994531f : -INFINITY;
+      p.lse[(static_cast<size_t>(b) * p.Hq + h) * p.T + row] = lse;
+    }
+    fence_proxy_async_smem();
+    named_barrier_sync(1 + t, kBM);
+    if (r == 0 && m0 + t * kBM < p.T) {
+      for (int c = 0; c < C::kChunks; ++c) tma_store_4d(&tmO, stage + c * C::kChunkBytes, c * 64, h, m0 + t * kBM, b);
+      tma_store_commit();
+      tma_store_wait_read0();
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+}  // namespace prefill
+}  // namespace attn

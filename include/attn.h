@@ -1,0 +1,147 @@
+/*
+ * attn.h - C ABI of the B200 (sm_100a) fused-attention library.
+ *
+ * The library computes softmax attention,  O = softmax(scale * Q K^T + mask) V,
+ * block by block with an online softmax, so that the T x S score matrix never
+ * reaches device memory.  That is the FlashAttention scheme of the page
+ * "Snelle attention-kernels en operatorfusie versnellen AI-modellen"
+ * (the-ai.news), section "FlashAttention-type aandacht en gepagineerde
+ * aandacht": queries, keys and values are processed per block; for each block
+ * a part of the scores is formed, the softmax statistics (running row maximum
+ * and running sum) are updated and the matching output is accumulated in
+ * on-chip memory.  The same section defines the paged KV cache served by
+ * paged_attn_decode: fixed-size blocks (16 tokens in its example) and a block
+ * table that maps every logical position to a physical block.
+ *
+ * Conventions shared by every entry point
+ * ----------------------------------------
+ *  - All tensor pointers are DEVICE pointers on the current CUDA device,
+ *    allocated, owned and freed by the caller.  The library never frees or
+ *    retains them beyond the call's completion on `stream`.
+ *  - bf16 tensors are passed as `void*` (IEEE bfloat16, row-major,
+ *    contiguous, 16-byte aligned base).  Float outputs are fp32.
+ *  - Every call is asynchronous on `stream` (a cudaStream_t; 0 = legacy
+ *    default stream) and performs no host<->device synchronisation.
+ *  - Return value: ATTN_OK (0) or a negative attn_status_t.  Argument errors
+ *    are detected on the host before anything is launched; nothing is written
+ *    to the outputs in that case.  There is no fallback path: an unsupported
+ *    shape returns ATTN_ERR_UNSUPPORTED.
+ *  - Device-side bounded waits: every wait inside a kernel gives up after a
+ *    time limit, records ATTN_DEVSTATUS_TIMEOUT in a device status word and
+ *    lets the kernel exit (the outputs of that call are then undefined).
+ *    attn_read_device_status() reads (and optionally clears) that word.
+ */
+#ifndef ATTN_B200_H
+#define ATTN_B200_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same type as cudaStream_t (struct CUstream_st*), declared here so that the
+ * header does not require the CUDA headers. */
+typedef struct CUstream_st* attn_stream_t;
+
+typedef enum {
+  ATTN_OK = 0,
+  ATTN_ERR_INVALID_ARG = -1, /* null pointer, negative size, Hq % Hkv != 0, bad scale ... */
+  ATTN_ERR_UNSUPPORTED = -2, /* valid but not implemented (head dim, block size, device) */
+  ATTN_ERR_CUDA = -3,        /* a CUDA runtime/driver call or a launch failed */
+  ATTN_ERR_TIMEOUT = -4      /* reported by attn_read_device_status() only */
+} attn_status_t;
+
+/* Bits of the device status word (see attn_read_device_status). */
+#define ATTN_DEVSTATUS_TIMEOUT 0x1
+
+/*
+ * attn_fwd - dense prefill attention with grouped-query heads.
+ *
+ *   q    [B, T, Hq,  d] bf16   queries
+ *   k    [B, S, Hkv, d] bf16   keys
+ *   v    [B, S, Hkv, d] bf16   values
+ *   o    [B, T, Hq,  d] bf16   output (written)
+ *   lse  [B, Hq, T]     fp32   per-row log-sum-exp of the scaled scores,
+ *                              natural log (written; may be NULL to skip)
+ *
+ *   Query head h reads key/value head h / (Hq / Hkv) (contiguous groups).
+ *   causal != 0: row i sees key j iff j <= i + (S - T) (bottom-right aligned;
+ *   the usual j <= i when T == S).  A row that sees no key gets O = 0 and
+ *   LSE = -inf.  scale multiplies Q K^T (1/sqrt(d) for standard attention).
+ *
+ *   Supported: d in {64, 128}; Hq % Hkv == 0; B, T, S >= 0 (T == 0 or
+ *   B == 0 is a no-op); sm_100 device.  Pointers 16-byte aligned.
+ *   Errors: ATTN_ERR_INVALID_ARG for null pointers, negative sizes,
+ *   Hq/Hkv <= 0, Hq % Hkv != 0, non-finite or non-positive scale;
+ *   ATTN_ERR_UNSUPPORTED for other head dims, unaligned pointers or a
+ *   non-sm_100 device; ATTN_ERR_CUDA if a launch fails.
+ */
+int attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
+             int B, int Hq, int Hkv, int T, int S, int d, int causal, float scale,
+             attn_stream_t stream);
+
+/*
+ * paged_attn_decode - one query token per sequence against a paged KV cache.
+ *
+ *   q            [B, Hq, d]                         bf16
+ *   k_cache      [num_blocks, block_size, Hkv, d]   bf16  (pool of physical blocks)
+ *   v_cache      [num_blocks, block_size, Hkv, d]   bf16
+ *   block_table  [B, max_blocks] int32: physical block of logical block j of
+ *                sequence b.  Only entries j < ceil(seq_lens[b]/block_size)
+ *                are read; they must be valid block ids of the pool.
+ *   seq_lens     [B] int32: cached tokens of each sequence (0 allowed, which
+ *                gives O = 0).  Must not exceed max_blocks * block_size.
+ *   o            [B, Hq, d] bf16 (written)
+ *
+ *   The query of sequence b sits at position seq_lens[b]-1 and sees every
+ *   cached token, scale = 1/sqrt(d).  Query head h reads kv head
+ *   h / (Hq / Hkv).
+ *
+ *   num_splits: the logical blocks of each sequence are cut into ranges of
+ *   ceil(max_blocks / num_splits) blocks, each handled by its own CTA, and
+ *   the partial results are merged with a log-sum-exp combine.  num_splits
+ *   <= 0 picks a value that fills the GPU.  The result does not depend on
+ *   the physical placement of the blocks (bit-identical for any permutation
+ *   of block ids with the same num_splits).
+ *
+ *   Workspace: partial outputs (num_splits * B * Hq * (d + 1) fp32) come from
+ *   a library-owned, stream-ordered memory pool (cudaMallocFromPoolAsync /
+ *   cudaFreeAsync on `stream`).
+ *
+ *   Supported: d in {64, 128}; block_size == 16; 1 <= Hq/Hkv <= 8;
+ *   sm_100 device; 16-byte aligned q, caches and o.
+ *   Errors: as attn_fwd; ATTN_ERR_INVALID_ARG also for max_blocks <= 0 when
+ *   B > 0.
+ */
+int paged_attn_decode(const void* q, const void* k_cache, const void* v_cache,
+                      const int32_t* block_table, const int32_t* seq_lens,
+                      int B, int Hq, int Hkv, int d, int block_size, int max_blocks,
+                      int num_splits, void* o, attn_stream_t stream);
+
+/*
+ * attn_check_support - initialisation-time compatibility check of `device`,
+ * in the spirit of the backend check at start-up described in the same
+ * section of the page (an incompatible backend is reported as an error at
+ * initialisation instead of failing later).  Returns ATTN_OK when the device
+ * is an sm_100 part this library was built for, ATTN_ERR_UNSUPPORTED when it
+ * is not, ATTN_ERR_CUDA when the device cannot be queried.
+ */
+int attn_check_support(int device);
+
+/* Static, human-readable name of a status code (never NULL). */
+const char* attn_status_string(int status);
+
+/*
+ * attn_read_device_status - copy the device status word of the current
+ * device into *out (synchronous: waits for the device) and clear it when
+ * `clear` != 0.  Bit ATTN_DEVSTATUS_TIMEOUT means a bounded wait inside a
+ * kernel gave up.  Returns ATTN_OK or ATTN_ERR_CUDA / ATTN_ERR_INVALID_ARG.
+ */
+int attn_read_device_status(int* out, int clear);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* ATTN_B200_H */
