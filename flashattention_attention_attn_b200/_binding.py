@@ -40,6 +40,8 @@ def library() -> ctypes.CDLL:
         lib.paged_attn_decode.argtypes = [vp, vp, vp, vp, vp, c_int, c_int, c_int, c_int, c_int, c_int, c_int,
                                           vp, vp]
         lib.paged_attn_decode.restype = c_int
+        lib.paged_attn_decode_noalloc.argtypes = lib.paged_attn_decode.argtypes
+        lib.paged_attn_decode_noalloc.restype = c_int
         lib.attn_check_support.argtypes = [c_int]
         lib.attn_check_support.restype = c_int
         lib.attn_status_string.argtypes = [c_int]
@@ -89,6 +91,18 @@ def paged_attn_decode(q, k_cache, v_cache, block_table, seq_lens, B, Hq, Hkv, d,
                                      int(num_splits), _ptr(o), _stream(stream))
     if rc != ATTN_OK:
         raise AttnError(rc, "paged_attn_decode")
+
+
+def paged_attn_decode_noalloc(q, k_cache, v_cache, block_table, seq_lens, B, Hq, Hkv, d, block_size,
+                              max_blocks, num_splits, o, stream=None) -> None:
+    """paged_attn_decode with its split partials in the library's fixed
+    scratch array: for callers that must not allocate during the call (see
+    attn.h for the size limit and the sharing rules)."""
+    rc = library().paged_attn_decode_noalloc(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_table),
+                                             _ptr(seq_lens), int(B), int(Hq), int(Hkv), int(d), int(block_size),
+                                             int(max_blocks), int(num_splits), _ptr(o), _stream(stream))
+    if rc != ATTN_OK:
+        raise AttnError(rc, "paged_attn_decode_noalloc")
 
 
 def attn_check_support(device: int = 0) -> int:

@@ -348,3 +348,128 @@ extern "C" int attn_read_device_status(int* out, int clear) {
   }
   return ATTN_OK;
 }
+
+// ---------------------------------------------------------------------------
+// paged_attn_decode_noalloc: the same kernels with their split partials in a
+// fixed scratch array compiled into the library instead of pool memory.
+// ---------------------------------------------------------------------------
+namespace attn {
+namespace {
+
+// Scratch for the split partials of paged_attn_decode_noalloc.  In host code
+// this name is only a stand-in for the device array; its device address is
+// looked up with cudaGetSymbolAddress once per device.
+static __device__ __align__(256) unsigned char g_noalloc_scratch[ATTN_NOALLOC_SCRATCH_BYTES];
+
+struct NoAllocState {
+  bool ready = false;
+  void* scratch = nullptr;  // device address of g_noalloc_scratch on this device
+};
+NoAllocState g_noalloc[kMaxDevices];
+
+// Once per device, with that device current: shared-memory limits of the
+// decode kernels and the scratch array's device address.  No allocation.
+int prepare_noalloc(int dev, void** scratch) {
+  std::lock_guard<std::mutex> lock(g_mu);
+  NoAllocState& na = g_noalloc[dev];
+  if (!na.ready) {
+    if (cudaFuncSetAttribute(reinterpret_cast<const void*>(decode::paged_decode_split<64>),
+                             cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(decode::smem_bytes<64>())) != cudaSuccess ||
+        cudaFuncSetAttribute(reinterpret_cast<const void*>(decode::paged_decode_split<128>),
+                             cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(decode::smem_bytes<128>())) != cudaSuccess) {
+      cudaGetLastError();
+      return ATTN_ERR_CUDA;
+    }
+    void* ptr = nullptr;
+    if (cudaGetSymbolAddress(&ptr, g_noalloc_scratch) != cudaSuccess || ptr == nullptr) {
+      cudaGetLastError();
+      return ATTN_ERR_CUDA;
+    }
+    na.scratch = ptr;
+    na.ready = true;
+  }
+  *scratch = na.scratch;
+  return ATTN_OK;
+}
+
+template <int D>
+int launch_decode_noalloc(const void* q, const void* kc, const void* vc, const int32_t* table,
+                          const int32_t* lens, int B, int Hq, int Hkv, int max_blocks, int num_splits, void* o,
+                          cudaStream_t stream, int sms, void* scratch) {
+  const int groups = (Hkv + decode::kKH - 1) / decode::kKH;
+  if (num_splits <= 0) num_splits = auto_splits(B, groups, max_blocks, sms);
+  if (num_splits > max_blocks) num_splits = max_blocks;
+  const int chunk = (max_blocks + num_splits - 1) / num_splits;
+  num_splits = (max_blocks + chunk - 1) / chunk;
+  if (num_splits > 65535 || groups > 65535 || B > 65535) return ATTN_ERR_UNSUPPORTED;
+  const size_t rows = static_cast<size_t>(num_splits) * B * Hq;
+  if (num_splits > 1 && rows * (D + 1) * sizeof(float) > ATTN_NOALLOC_SCRATCH_BYTES) return ATTN_ERR_UNSUPPORTED;
+  CUtensorMap mk, mv;
+  if (make_map_pool(&mk, kc, Hkv, D) || make_map_pool(&mv, vc, Hkv, D)) return ATTN_ERR_CUDA;
+
+  decode::Params p;
+  p.q = static_cast<const __nv_bfloat16*>(q);
+  p.block_table = table;
+  p.seq_lens = lens;
+  p.o = static_cast<__nv_bfloat16*>(o);
+  p.part_o = num_splits > 1 ? static_cast<float*>(scratch) : nullptr;
+  p.part_lse = num_splits > 1 ? static_cast<float*>(scratch) + rows * D : nullptr;
+  p.B = B;
+  p.Hq = Hq;
+  p.Hkv = Hkv;
+  p.max_blocks = max_blocks;
+  p.num_splits = num_splits;
+  p.chunk = chunk;
+  p.scale_log2 = (1.0f / std::sqrt(static_cast<float>(D))) * 1.4426950408889634f;
+
+  dim3 grid(num_splits, groups, B);
+  decode::paged_decode_split<D><<<grid, (decode::kKH + 1) * 32, decode::smem_bytes<D>(), stream>>>(mk, mv, p);
+  int rc = launch_status();
+  if (rc == ATTN_OK && num_splits > 1) {
+    dim3 cgrid(Hq, B, D / 32);
+    decode::lse_combine<D><<<cgrid, 128, 0, stream>>>(p.part_o, p.part_lse, lens, p.o, B, Hq, num_splits, chunk);
+    rc = launch_status();
+  }
+  return rc;
+}
+
+}  // namespace
+}  // namespace attn
+
+extern "C" int paged_attn_decode_noalloc(const void* q, const void* k_cache, const void* v_cache,
+                                         const int32_t* block_table, const int32_t* seq_lens, int B, int Hq,
+                                         int Hkv, int d, int block_size, int max_blocks, int num_splits, void* o,
+                                         attn_stream_t stream_) {
+  cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+  if (B < 0 || Hq <= 0 || Hkv <= 0 || d <= 0 || block_size <= 0) return ATTN_ERR_INVALID_ARG;
+  if (Hq % Hkv != 0) return ATTN_ERR_INVALID_ARG;
+  if (B == 0) return ATTN_OK;
+  if (max_blocks <= 0) return ATTN_ERR_INVALID_ARG;
+  if (q == nullptr || k_cache == nullptr || v_cache == nullptr || block_table == nullptr || seq_lens == nullptr ||
+      o == nullptr)
+    return ATTN_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return ATTN_ERR_UNSUPPORTED;
+  if (block_size != decode::kBlock) return ATTN_ERR_UNSUPPORTED;
+  if (Hq / Hkv > 8) return ATTN_ERR_UNSUPPORTED;
+  if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(o)) return ATTN_ERR_UNSUPPORTED;
+  if ((reinterpret_cast<uintptr_t>(block_table) & 3u) || (reinterpret_cast<uintptr_t>(seq_lens) & 3u))
+    return ATTN_ERR_UNSUPPORTED;
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess) {
+    cudaGetLastError();
+    return ATTN_ERR_CUDA;
+  }
+  DeviceState* st = nullptr;
+  int rc = probe_device(dev, &st);
+  if (rc != ATTN_OK) return rc;
+  void* scratch = nullptr;
+  rc = prepare_noalloc(dev, &scratch);
+  if (rc != ATTN_OK) return rc;
+  if (d == 64)
+    return launch_decode_noalloc<64>(q, k_cache, v_cache, block_table, seq_lens, B, Hq, Hkv, max_blocks,
+                                     num_splits, o, stream, st->sms, scratch);
+  return launch_decode_noalloc<128>(q, k_cache, v_cache, block_table, seq_lens, B, Hq, Hkv, max_blocks,
+                                    num_splits, o, stream, st->sms, scratch);
+}

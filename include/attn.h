@@ -140,6 +140,44 @@ const char* attn_status_string(int status);
  */
 int attn_read_device_status(int* out, int clear);
 
+/*
+ * paged_attn_decode_noalloc - paged_attn_decode for callers that must not
+ * allocate device memory during the call.
+ *
+ * The pages describe no such variant; it exists for integration only.  Some
+ * callers cannot let a library call cudaMalloc or draw from a memory pool:
+ * code running inside a pre-planned memory budget (an inference server that
+ * has already handed all free memory to its KV-cache pool), allocators that
+ * must not be re-entered from a callback, or callers that forbid any
+ * allocation on their hot path.  This entry point takes the same arguments
+ * and computes the same result as paged_attn_decode, but its split-KV
+ * partials live in one fixed scratch array compiled into the library
+ * (ATTN_NOALLOC_SCRATCH_BYTES per GPU, held by every GPU that loads the
+ * library until the process exits).  It calls no cudaMalloc, cudaFree or
+ * other allocating routine.
+ *
+ *   Limit: num_splits * B * Hq * (d + 1) * 4 bytes of partials (with the
+ *   split count after num_splits <= 0 is resolved and clamped) must not
+ *   exceed ATTN_NOALLOC_SCRATCH_BYTES; a larger request returns
+ *   ATTN_ERR_UNSUPPORTED before anything is launched.  With one split no
+ *   scratch is used.
+ *   First call on a device: it looks up the scratch array's device address
+ *   (cudaGetSymbolAddress, with that device current) and sets the kernels'
+ *   shared-memory limits; make that first call before any stream capture.
+ *   Sharing: every call on a device uses the same scratch array and it keeps
+ *   the previous call's contents (no part of it needs to start at zero: each
+ *   partial the merge reads is written earlier in the same call).  Calls that
+ *   can overlap on the GPU (different streams without ordering between them)
+ *   race on the scratch and give undefined results; serialise them.
+ *   Errors: as paged_attn_decode, plus the limit above.
+ */
+#define ATTN_NOALLOC_SCRATCH_BYTES (8u << 20)
+
+int paged_attn_decode_noalloc(const void* q, const void* k_cache, const void* v_cache,
+                              const int32_t* block_table, const int32_t* seq_lens,
+                              int B, int Hq, int Hkv, int d, int block_size, int max_blocks,
+                              int num_splits, void* o, attn_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif
