@@ -189,17 +189,44 @@ int launch_prefill(const void* q, const void* k, const void* v, void* o, float* 
   return launch_status();
 }
 
-// Splits chosen so that the CTAs of a batch whose sequences all reach
-// max_blocks fill the GPU about twice (2 CTAs of the decode kernel fit on
-// one SM), with at least 8 blocks per split.
+// Splits for num_splits <= 0.  The host does not know the sequence lengths
+// (they are on the device), so the choice assumes every sequence fills
+// max_blocks: a single sequence is cut into one wave of equal units (two
+// decode CTAs fit on an SM); a batch into about four waves, so that the
+// scheduler can balance units of unequal length.  At least 8 blocks per unit.
 int auto_splits(int B, int groups, int max_blocks, int sms) {
-  const long long units = static_cast<long long>(B) * groups;
-  const long long target = 4LL * sms;
-  long long splits = (target + units - 1) / units;
-  const long long max_splits = (max_blocks + 7) / 8;
-  if (splits > max_splits) splits = max_splits;
-  if (splits < 1) splits = 1;
-  return static_cast<int>(splits);
+  const long long slots = 2LL * sms;
+  const long long waves = (B == 1) ? 1 : 4;
+  const long long blocks = static_cast<long long>(B) * groups * max_blocks;
+  long long chunk = (blocks + waves * slots - 1) / (waves * slots);
+  if (chunk < 8) chunk = 8;
+  if (chunk > max_blocks) chunk = max_blocks;
+  return static_cast<int>((max_blocks + chunk - 1) / chunk);
+}
+
+// The LSE merge, launched as a programmatic dependent of the split kernel so
+// that its launch and prologue overlap the split kernel's tail.
+template <int D>
+int launch_combine(const decode::Params& p, const int32_t* lens, cudaStream_t stream) {
+  cudaLaunchConfig_t cfg;
+  std::memset(&cfg, 0, sizeof(cfg));
+  cfg.gridDim = dim3(p.Hq, p.B, 1);
+  cfg.blockDim = dim3(decode::kCombineWarps * 32, 1, 1);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  const float* po = p.part_o;
+  const float* pl = p.part_lse;
+  if (cudaLaunchKernelEx(&cfg, decode::lse_combine<D>, po, pl, lens, p.o, p.B, p.Hq, p.num_splits, p.chunk) !=
+      cudaSuccess) {
+    cudaGetLastError();
+    return ATTN_ERR_CUDA;
+  }
+  return ATTN_OK;
 }
 
 template <int D>
@@ -244,11 +271,7 @@ int launch_decode(const void* q, const void* kc, const void* vc, const int32_t* 
   dim3 grid(num_splits, groups, B);
   decode::paged_decode_split<D><<<grid, (decode::kKH + 1) * 32, decode::smem_bytes<D>(), stream>>>(mk, mv, p);
   int rc = launch_status();
-  if (rc == ATTN_OK && num_splits > 1) {
-    dim3 cgrid(Hq, B, D / 32);
-    decode::lse_combine<D><<<cgrid, 128, 0, stream>>>(p.part_o, p.part_lse, lens, p.o, B, Hq, num_splits, chunk);
-    rc = launch_status();
-  }
+  if (rc == ATTN_OK && num_splits > 1) rc = launch_combine<D>(p, lens, stream);
   if (ws != nullptr) cudaFreeAsync(ws, stream);
   return rc;
 }
@@ -427,11 +450,7 @@ int launch_decode_noalloc(const void* q, const void* kc, const void* vc, const i
   dim3 grid(num_splits, groups, B);
   decode::paged_decode_split<D><<<grid, (decode::kKH + 1) * 32, decode::smem_bytes<D>(), stream>>>(mk, mv, p);
   int rc = launch_status();
-  if (rc == ATTN_OK && num_splits > 1) {
-    dim3 cgrid(Hq, B, D / 32);
-    decode::lse_combine<D><<<cgrid, 128, 0, stream>>>(p.part_o, p.part_lse, lens, p.o, B, Hq, num_splits, chunk);
-    rc = launch_status();
-  }
+  if (rc == ATTN_OK && num_splits > 1) rc = launch_combine<D>(p, lens, stream);
   return rc;
 }
 

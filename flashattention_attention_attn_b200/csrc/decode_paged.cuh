@@ -82,6 +82,10 @@ __global__ void __launch_bounds__((kKH + 1) * 32, 2)
   extern __shared__ uint8_t smem_raw[];
   Smem<D>& sm = *reinterpret_cast<Smem<D>*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
 
+  // Let the combine kernel (launched as a programmatic dependent) be
+  // scheduled once every CTA of this grid has started; it waits for this
+  // grid's completion before it reads any partial.
+  asm volatile("griddepcontrol.launch_dependents;");
   const int split = blockIdx.x;
   const int hg = blockIdx.y;  // kv-head group
   const int b = blockIdx.z;
@@ -319,75 +323,98 @@ __global__ void __launch_bounds__((kKH + 1) * 32, 2)
 
 // Merge the split partials of every (sequence, query head):
 //   M = max_i lse_i,  O = sum_i e^{lse_i - M} o_i / sum_i e^{lse_i - M}.
-// One CTA of 128 threads per (query head, sequence, 32-column slice of d):
-// the 4 warps stride over the splits, lane c owns column 32*slice + c, and
-// the loop is unrolled so that several partial rows are in flight per warp.
+// One CTA of kCombineWarps warps per (query head, sequence).  Warp w merges
+// splits w, w + kCombineWarps, ... with a running maximum (so no separate
+// max pass), kUnroll rows in flight per lane; lane c owns D/32 consecutive
+// columns.  The per-warp results are then merged in shared memory in a
+// fixed order (deterministic).  Launched as a programmatic dependent of the
+// split kernel: everything before griddepcontrol.wait overlaps its tail.
+constexpr int kCombineWarps = 8;
+
 template <int D>
-__global__ void __launch_bounds__(128)
+__global__ void __launch_bounds__(kCombineWarps * 32)
     lse_combine(const float* __restrict__ part_o, const float* __restrict__ part_lse,
                 const int32_t* __restrict__ seq_lens, __nv_bfloat16* __restrict__ o, int B, int Hq,
                 int num_splits, int chunk) {
-  constexpr int kWarps = 4;
+  constexpr int kPer = D / 32;
   constexpr int kUnroll = 4;
+  constexpr float kLog2e = 1.4426950408889634f;
   const int h = blockIdx.x;
   const int b = blockIdx.y;
-  const int col = blockIdx.z * 32 + (threadIdx.x & 31);
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  __shared__ float red[kWarps][32];
-  __shared__ float wred[kWarps];
-  __shared__ float mred[kWarps];
+  __shared__ float s_acc[kCombineWarps][D];
+  __shared__ float s_m[kCombineWarps], s_w[kCombineWarps];
 
-  const int L = seq_lens[b];
+  const int L = seq_lens[b];  // an input of the call, not written by the split kernel
   const int nb = (L + kBlock - 1) / kBlock;
   const int nsp = min(num_splits, (nb + chunk - 1) / chunk);  // splits holding data
   __nv_bfloat16* out = o + (static_cast<size_t>(b) * Hq + h) * D;
+  asm volatile("griddepcontrol.wait;" ::: "memory");
   if (nsp <= 0) {
-    if (warp == 0) out[col] = __float2bfloat16_rn(0.f);
+    if (threadIdx.x < D) out[threadIdx.x] = __float2bfloat16_rn(0.f);
     return;
   }
   const size_t stride = static_cast<size_t>(B) * Hq;  // rows between splits
   const size_t head = static_cast<size_t>(b) * Hq + h;
 
-  float mx = -INFINITY;
-  for (int i = threadIdx.x; i < nsp; i += kWarps * 32) mx = fmaxf(mx, part_lse[i * stride + head]);
+  float m = -INFINITY, wsum = 0.f;  // log2-domain running max and weight sum
+  float acc[kPer];
 #pragma unroll
-  for (int off = 16; off > 0; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
-  if (lane == 0) mred[warp] = mx;
-  __syncthreads();
-  mx = fmaxf(fmaxf(mred[0], mred[1]), fmaxf(mred[2], mred[3]));
-
-  constexpr float kLog2e = 1.4426950408889634f;
-  float acc = 0.f, wsum = 0.f;
-  int i = warp;
-  for (; i + (kUnroll - 1) * kWarps < nsp; i += kUnroll * kWarps) {
-    float lv[kUnroll], ov[kUnroll];
+  for (int e = 0; e < kPer; ++e) acc[e] = 0.f;
+  for (int i0 = warp; i0 < nsp; i0 += kUnroll * kCombineWarps) {
+    float lv[kUnroll];
+    float ov[kUnroll][kPer];
 #pragma unroll
     for (int u = 0; u < kUnroll; ++u) {
-      const size_t row = (i + u * kWarps) * stride + head;
-      lv[u] = part_lse[row];
-      ov[u] = part_o[row * D + col];
+      const int i = i0 + u * kCombineWarps;
+      const size_t row = static_cast<size_t>(min(i, nsp - 1)) * stride + head;
+      lv[u] = (i < nsp) ? part_lse[row] * kLog2e : -INFINITY;
+      const float* src = part_o + row * D + lane * kPer;
+      if constexpr (kPer == 4) {
+        const float4 v = *reinterpret_cast<const float4*>(src);
+        ov[u][0] = v.x, ov[u][1] = v.y, ov[u][2] = v.z, ov[u][3] = v.w;
+      } else {
+        const float2 v = *reinterpret_cast<const float2*>(src);
+        ov[u][0] = v.x, ov[u][1] = v.y;
+      }
     }
+    float mx = m;
+#pragma unroll
+    for (int u = 0; u < kUnroll; ++u) mx = fmaxf(mx, lv[u]);
+    const float sc = ex2_approx(m - mx);  // m = -inf on the first round: 0
+    wsum *= sc;
+#pragma unroll
+    for (int e = 0; e < kPer; ++e) acc[e] *= sc;
 #pragma unroll
     for (int u = 0; u < kUnroll; ++u) {
-      const float w = ex2_approx((lv[u] - mx) * kLog2e);
-      acc = fmaf(w, ov[u], acc);
+      const float w = ex2_approx(lv[u] - mx);  // 0 for rows past nsp
       wsum += w;
+#pragma unroll
+      for (int e = 0; e < kPer; ++e) acc[e] = fmaf(w, ov[u][e], acc[e]);
     }
+    m = mx;
   }
-  for (; i < nsp; i += kWarps) {
-    const size_t row = i * stride + head;
-    const float w = ex2_approx((part_lse[row] - mx) * kLog2e);
-    acc = fmaf(w, part_o[row * D + col], acc);
-    wsum += w;
+#pragma unroll
+  for (int e = 0; e < kPer; ++e) s_acc[warp][lane * kPer + e] = acc[e];
+  if (lane == 0) {
+    s_m[warp] = m;
+    s_w[warp] = wsum;
   }
-  red[warp][lane] = acc;
-  if (lane == 0) wred[warp] = wsum;
   __syncthreads();
-  if (warp == 0) {
-    const float tot = (red[0][lane] + red[1][lane]) + (red[2][lane] + red[3][lane]);
-    const float ws = (wred[0] + wred[1]) + (wred[2] + wred[3]);
-    out[col] = __float2bfloat16_rn(tot / ws);
+  if (threadIdx.x < D) {
+    const int c = threadIdx.x;
+    float M = -INFINITY;
+#pragma unroll
+    for (int w = 0; w < kCombineWarps; ++w) M = fmaxf(M, s_m[w]);
+    float tot = 0.f, ws = 0.f;
+#pragma unroll
+    for (int w = 0; w < kCombineWarps; ++w) {
+      const float f = ex2_approx(s_m[w] - M);  // warps without rows: -inf -> 0
+      tot = fmaf(f, s_acc[w][c], tot);
+      ws = fmaf(f, s_w[w], ws);
+    }
+    out[c] = __float2bfloat16_rn(tot / ws);
   }
 }
 

@@ -171,7 +171,7 @@ int attn_read_device_status(int* out, int clear);
  *   race on the scratch and give undefined results; serialise them.
  *   Errors: as paged_attn_decode, plus the limit above.
  */
-#define ATTN_NOALLOC_SCRATCH_BYTES (8u << 20)
+#define ATTN_NOALLOC_SCRATCH_BYTES (16u << 20)
 
 int paged_attn_decode_noalloc(const void* q, const void* k_cache, const void* v_cache,
                               const int32_t* block_table, const int32_t* seq_lens,

@@ -42,6 +42,6 @@ def test_noalloc_rejects_partials_beyond_the_scratch_size():
     spec = inputs.DecodeSpec(B=64, Hq=32, Hkv=8, d=128, block_size=16, max_blocks=256, ctx_lo=16, ctx_hi=64,
                              seed=3)
     inp = inputs.make_paged(spec)
-    with pytest.raises(fa.AttnError) as err:  # 256 splits * 64 * 32 rows * 129 floats > 8 MiB
+    with pytest.raises(fa.AttnError) as err:  # 256 splits * 64 * 32 rows * 129 floats > 16 MiB
         _run(fa.paged_attn_decode_noalloc, inp, 256)
     assert err.value.status == -2
