@@ -198,7 +198,7 @@ def main():
     import torch.distributed as dist
 
     import flashattention_attention_attn_b200 as fa
-    from flashattention_attention_attn_b200 import build as _build, inputs, workloads
+    from flashattention_attention_attn_b200 import build as _build, dist_util, inputs, workloads
 
     if not os.path.exists(_build.LIB_PATH):
         _build.build()
@@ -213,8 +213,8 @@ def main():
     ps = inputs.WORKLOADS[pname]
     ds = inputs.WORKLOADS[dname]
     # weak scaling: every rank runs its own batch (different seeds), no exchange
-    q, k, v = inputs.make_prefill(ps, seed=ps.seed + 100 * rank)
-    dinp = inputs.make_paged(ds, seed=ds.seed + 100 * rank)
+    q, k, v = inputs.make_prefill(ps, seed=dist_util.rank_seed(ps.seed, rank))
+    dinp = inputs.make_paged(ds, seed=dist_util.rank_seed(ds.seed, rank))
     dq, dk, dv = q.to(dev), k.to(dev), v.to(dev)
     o = torch.empty_like(dq)
     lse = torch.empty(ps.B, ps.Hq, ps.T, device=dev, dtype=torch.float32)
@@ -270,10 +270,7 @@ def main():
     t_pre = sum(ev[i][0].elapsed_time(ev[i][1]) for i in range(K)) / K
     t_dec = sum(ev[i][1].elapsed_time(ev[i][2]) for i in range(K)) / K
     ms_step = total_ms / K
-    if world > 1:
-        t = torch.tensor([ms_step, t_pre, t_dec], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms_step, t_pre, t_dec = t.tolist()
+    ms_step, t_pre, t_dec = dist_util.max_over_ranks([ms_step, t_pre, t_dec], device=dev)
 
     ideal_pre = flops / (peaks["bf16_tflops"] * 1e12)
     ideal_dec = dbytes / (peaks["hbm_gbs"] * 1e9)
@@ -308,10 +305,7 @@ def main():
         e1.record(stream)
         torch.cuda.synchronize()
         e2e_ms = e0.elapsed_time(e1) / args.e2e_steps
-        if world > 1:
-            t = torch.tensor([e2e_ms], device=dev)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            e2e_ms = t.item()
+        (e2e_ms,) = dist_util.max_over_ranks([e2e_ms], device=dev)
         e2e = {"value": 100.0 * world * ideal / (e2e_ms * 1e-3), "unit": UNIT, "h2d_bytes_per_step": int(h2d),
                "d2h_bytes_per_step": int(d2h), "ms_per_step": e2e_ms}
 
