@@ -205,13 +205,16 @@ int auto_splits(int B, int groups, int max_blocks, int sms) {
 }
 
 // The LSE merge, launched as a programmatic dependent of the split kernel so
-// that its launch and prologue overlap the split kernel's tail.
-template <int D>
-int launch_combine(const decode::Params& p, const int32_t* lens, cudaStream_t stream) {
+// that its launch and prologue overlap the split kernel's tail.  WPR warps
+// per (sequence, head) row: about 8 splits per warp, at most 16 warps.
+template <int D, int WPR>
+int launch_combine_wpr(const decode::Params& p, const int32_t* lens, cudaStream_t stream) {
+  using Shape = decode::CombineShape<WPR>;
+  const long long rows = static_cast<long long>(p.B) * p.Hq;
   cudaLaunchConfig_t cfg;
   std::memset(&cfg, 0, sizeof(cfg));
-  cfg.gridDim = dim3(p.Hq, p.B, 1);
-  cfg.blockDim = dim3(decode::kCombineWarps * 32, 1, 1);
+  cfg.gridDim = dim3(static_cast<unsigned>((rows + Shape::kRows - 1) / Shape::kRows), 1, 1);
+  cfg.blockDim = dim3(Shape::kWarps * 32, 1, 1);
   cfg.dynamicSmemBytes = 0;
   cfg.stream = stream;
   cudaLaunchAttribute attr[1];
@@ -221,12 +224,23 @@ int launch_combine(const decode::Params& p, const int32_t* lens, cudaStream_t st
   cfg.numAttrs = 1;
   const float* po = p.part_o;
   const float* pl = p.part_lse;
-  if (cudaLaunchKernelEx(&cfg, decode::lse_combine<D>, po, pl, lens, p.o, p.B, p.Hq, p.num_splits, p.chunk) !=
-      cudaSuccess) {
+  if (cudaLaunchKernelEx(&cfg, decode::lse_combine<D, WPR>, po, pl, lens, p.o, p.B, p.Hq, p.num_splits,
+                         p.chunk) != cudaSuccess) {
     cudaGetLastError();
     return ATTN_ERR_CUDA;
   }
   return ATTN_OK;
+}
+
+template <int D>
+int launch_combine(const decode::Params& p, const int32_t* lens, cudaStream_t stream) {
+  const int per_warp = 8;
+  const int need = (p.num_splits + per_warp - 1) / per_warp;
+  if (need <= 1) return launch_combine_wpr<D, 1>(p, lens, stream);
+  if (need <= 2) return launch_combine_wpr<D, 2>(p, lens, stream);
+  if (need <= 4) return launch_combine_wpr<D, 4>(p, lens, stream);
+  if (need <= 8) return launch_combine_wpr<D, 8>(p, lens, stream);
+  return launch_combine_wpr<D, 16>(p, lens, stream);
 }
 
 template <int D>

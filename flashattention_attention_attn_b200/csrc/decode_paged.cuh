@@ -323,52 +323,57 @@ __global__ void __launch_bounds__((kKH + 1) * 32, 2)
 
 // Merge the split partials of every (sequence, query head):
 //   M = max_i lse_i,  O = sum_i e^{lse_i - M} o_i / sum_i e^{lse_i - M}.
-// One CTA of kCombineWarps warps per (query head, sequence).  Warp w merges
-// splits w, w + kCombineWarps, ... with a running maximum (so no separate
-// max pass), kUnroll rows in flight per lane; lane c owns D/32 consecutive
-// columns.  The per-warp results are then merged in shared memory in a
+// WPR warps merge one (sequence, query head) row; a CTA holds
+// max(8, WPR) warps, i.e. max(1, 8 / WPR) rows, so that few splits give one
+// wave of CTAs and many splits spread each row over up to 16 warps.  Warp w
+// of a row takes splits w, w + WPR, ... with a running maximum (no separate
+// max pass) and kUnroll rows in flight per lane; lane c owns D/32
+// consecutive columns.  The row's warps are merged in shared memory in a
 // fixed order (deterministic).  Launched as a programmatic dependent of the
 // split kernel: everything before griddepcontrol.wait overlaps its tail.
-constexpr int kCombineWarps = 8;
+template <int WPR>
+struct CombineShape {
+  static constexpr int kWarps = WPR > 8 ? WPR : 8;
+  static constexpr int kRows = kWarps / WPR;
+};
 
-template <int D>
-__global__ void __launch_bounds__(kCombineWarps * 32)
+template <int D, int WPR>
+__global__ void __launch_bounds__(CombineShape<WPR>::kWarps * 32)
     lse_combine(const float* __restrict__ part_o, const float* __restrict__ part_lse,
                 const int32_t* __restrict__ seq_lens, __nv_bfloat16* __restrict__ o, int B, int Hq,
                 int num_splits, int chunk) {
+  using Shape = CombineShape<WPR>;
   constexpr int kPer = D / 32;
   constexpr int kUnroll = 4;
   constexpr float kLog2e = 1.4426950408889634f;
-  const int h = blockIdx.x;
-  const int b = blockIdx.y;
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  __shared__ float s_acc[kCombineWarps][D];
-  __shared__ float s_m[kCombineWarps], s_w[kCombineWarps];
+  const int local_row = warp / WPR;
+  const int sub = warp % WPR;
+  const int row_id = blockIdx.x * Shape::kRows + local_row;  // = b * Hq + h
+  const bool live = row_id < B * Hq;
+  __shared__ float s_acc[Shape::kWarps][D];
+  __shared__ float s_m[Shape::kWarps], s_w[Shape::kWarps];
 
-  const int L = seq_lens[b];  // an input of the call, not written by the split kernel
-  const int nb = (L + kBlock - 1) / kBlock;
-  const int nsp = min(num_splits, (nb + chunk - 1) / chunk);  // splits holding data
-  __nv_bfloat16* out = o + (static_cast<size_t>(b) * Hq + h) * D;
-  asm volatile("griddepcontrol.wait;" ::: "memory");
-  if (nsp <= 0) {
-    if (threadIdx.x < D) out[threadIdx.x] = __float2bfloat16_rn(0.f);
-    return;
+  int nsp = 0;
+  if (live) {
+    const int L = seq_lens[row_id / Hq];  // an input of the call, not written by the split kernel
+    nsp = min(num_splits, (((L + kBlock - 1) / kBlock) + chunk - 1) / chunk);  // splits holding data
   }
+  asm volatile("griddepcontrol.wait;" ::: "memory");
   const size_t stride = static_cast<size_t>(B) * Hq;  // rows between splits
-  const size_t head = static_cast<size_t>(b) * Hq + h;
 
   float m = -INFINITY, wsum = 0.f;  // log2-domain running max and weight sum
   float acc[kPer];
 #pragma unroll
   for (int e = 0; e < kPer; ++e) acc[e] = 0.f;
-  for (int i0 = warp; i0 < nsp; i0 += kUnroll * kCombineWarps) {
+  for (int i0 = sub; i0 < nsp; i0 += kUnroll * WPR) {
     float lv[kUnroll];
     float ov[kUnroll][kPer];
 #pragma unroll
     for (int u = 0; u < kUnroll; ++u) {
-      const int i = i0 + u * kCombineWarps;
-      const size_t row = static_cast<size_t>(min(i, nsp - 1)) * stride + head;
+      const int i = i0 + u * WPR;
+      const size_t row = static_cast<size_t>(min(i, nsp - 1)) * stride + row_id;
       lv[u] = (i < nsp) ? part_lse[row] * kLog2e : -INFINITY;
       const float* src = part_o + row * D + lane * kPer;
       if constexpr (kPer == 4) {
@@ -395,26 +400,47 @@ __global__ void __launch_bounds__(kCombineWarps * 32)
     }
     m = mx;
   }
+  if constexpr (WPR == 1) {
+    if (!live) return;
+    __nv_bfloat16* out = o + static_cast<size_t>(row_id) * D + lane * kPer;
+    const float inv = (nsp > 0) ? 1.0f / wsum : 0.f;  // empty sequence: O = 0
 #pragma unroll
-  for (int e = 0; e < kPer; ++e) s_acc[warp][lane * kPer + e] = acc[e];
-  if (lane == 0) {
-    s_m[warp] = m;
-    s_w[warp] = wsum;
-  }
-  __syncthreads();
-  if (threadIdx.x < D) {
-    const int c = threadIdx.x;
+    for (int e = 0; e < kPer; ++e) out[e] = __float2bfloat16_rn(acc[e] * inv);
+    return;
+  } else {
+#pragma unroll
+    for (int e = 0; e < kPer; ++e) s_acc[warp][lane * kPer + e] = acc[e];
+    if (lane == 0) {
+      s_m[warp] = m;
+      s_w[warp] = wsum;
+    }
+    __syncthreads();
+    if (!live || sub != 0) return;
+    __nv_bfloat16* out = o + static_cast<size_t>(row_id) * D + lane * kPer;
+    if (nsp == 0) {  // empty sequence: O = 0
+#pragma unroll
+      for (int e = 0; e < kPer; ++e) out[e] = __float2bfloat16_rn(0.f);
+      return;
+    }
+    // the first warp of the row merges its WPR warps
+    const int w0 = local_row * WPR;
     float M = -INFINITY;
 #pragma unroll
-    for (int w = 0; w < kCombineWarps; ++w) M = fmaxf(M, s_m[w]);
-    float tot = 0.f, ws = 0.f;
+    for (int w = 0; w < WPR; ++w) M = fmaxf(M, s_m[w0 + w]);
+    float ws = 0.f;
+    float tot[kPer];
 #pragma unroll
-    for (int w = 0; w < kCombineWarps; ++w) {
-      const float f = ex2_approx(s_m[w] - M);  // warps without rows: -inf -> 0
-      tot = fmaf(f, s_acc[w][c], tot);
-      ws = fmaf(f, s_w[w], ws);
+    for (int e = 0; e < kPer; ++e) tot[e] = 0.f;
+#pragma unroll
+    for (int w = 0; w < WPR; ++w) {
+      const float f = ex2_approx(s_m[w0 + w] - M);  // warps without rows: -inf -> 0
+      ws = fmaf(f, s_w[w0 + w], ws);
+#pragma unroll
+      for (int e = 0; e < kPer; ++e) tot[e] = fmaf(f, s_acc[w0 + w][lane * kPer + e], tot[e]);
     }
-    out[c] = __float2bfloat16_rn(tot / ws);
+    const float inv = 1.0f / ws;
+#pragma unroll
+    for (int e = 0; e < kPer; ++e) out[e] = __float2bfloat16_rn(tot[e] * inv);
   }
 }
 
