@@ -48,6 +48,8 @@ def library() -> ctypes.CDLL:
         lib.attn_status_string.restype = ctypes.c_char_p
         lib.attn_read_device_status.argtypes = [ctypes.POINTER(c_int), c_int]
         lib.attn_read_device_status.restype = c_int
+        lib.attn_selftest_bounded_wait.argtypes = [vp]
+        lib.attn_selftest_bounded_wait.restype = c_int
         _lib = lib
     return _lib
 
@@ -115,3 +117,11 @@ def attn_read_device_status(clear: bool = True) -> int:
     if rc != ATTN_OK:
         raise AttnError(rc, "attn_read_device_status")
     return int(out.value)
+
+
+def attn_selftest_bounded_wait(stream=None) -> None:
+    """Launch the bounded-wait self test (see attn.h); read the outcome with
+    attn_read_device_status()."""
+    rc = library().attn_selftest_bounded_wait(_stream(stream))
+    if rc != ATTN_OK:
+        raise AttnError(rc, "attn_selftest_bounded_wait")

@@ -275,7 +275,17 @@ int launch_decode(const void* q, const void* kc, const void* vc, const int32_t* 
   if (num_splits > 1) {
     const size_t rows = static_cast<size_t>(num_splits) * B * Hq;
     const size_t bytes = rows * D * sizeof(float) + rows * sizeof(float);
-    if (cudaMallocFromPoolAsync(&ws, bytes, st->pool, stream) != cudaSuccess) {
+    // Outside capture the workspace comes from the library's pool; inside a
+    // stream capture from cudaMallocAsync, which becomes a graph memory node.
+    cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
+    if (cudaStreamIsCapturing(stream, &cap) != cudaSuccess) {
+      cudaGetLastError();
+      return ATTN_ERR_CUDA;
+    }
+    const cudaError_t ae = (cap == cudaStreamCaptureStatusActive)
+                               ? cudaMallocAsync(&ws, bytes, stream)
+                               : cudaMallocFromPoolAsync(&ws, bytes, st->pool, stream);
+    if (ae != cudaSuccess) {
       cudaGetLastError();
       return ATTN_ERR_CUDA;
     }
@@ -366,6 +376,28 @@ extern "C" const char* attn_status_string(int status) {
     default:
       return "unknown status";
   }
+}
+
+namespace attn {
+namespace {
+// One thread waits on a barrier that expects one arrival that never comes.
+__global__ void selftest_bounded_wait_kernel() {
+  __shared__ uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    abort_flag = 0;
+    fence_mbarrier_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) mbar_wait(&bar, 0, &abort_flag);  // gives up after the limit
+}
+}  // namespace
+}  // namespace attn
+
+extern "C" int attn_selftest_bounded_wait(attn_stream_t stream_) {
+  attn::selftest_bounded_wait_kernel<<<1, 32, 0, reinterpret_cast<cudaStream_t>(stream_)>>>();
+  return attn::launch_status();
 }
 
 extern "C" int attn_read_device_status(int* out, int clear) {

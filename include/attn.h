@@ -141,6 +141,17 @@ const char* attn_status_string(int status);
 int attn_read_device_status(int* out, int clear);
 
 /*
+ * attn_selftest_bounded_wait - exercise the give-up path of the kernels'
+ * bounded waits.  Launches one CTA on `stream` that waits, with the same
+ * wait routine and the same time limit (about 1 s) as the attention kernels,
+ * on an mbarrier that nothing ever arrives on.  The wait gives up, sets
+ * ATTN_DEVSTATUS_TIMEOUT in the device status word and the kernel exits; the
+ * CUDA context stays usable.  Read the result with attn_read_device_status().
+ * Returns ATTN_OK when the launch succeeded.
+ */
+int attn_selftest_bounded_wait(attn_stream_t stream);
+
+/*
  * paged_attn_decode_noalloc - paged_attn_decode for callers that must not
  * allocate device memory during the call.
  *

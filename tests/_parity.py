@@ -29,9 +29,10 @@ def check_close(o_gpu, o_ref, lse_gpu=None, lse_ref=None, what=""):
     if lse_gpu is not None:
         lg = np.asarray(lse_gpu, dtype=np.float64)
         lr = np.asarray(lse_ref, dtype=np.float64)
-        both_inf = np.isneginf(lg) & np.isneginf(lr)
         assert np.array_equal(np.isneginf(lg), np.isneginf(lr)), f"{what}: -inf pattern of LSE differs"
-        dl = np.abs(np.where(both_inf, 0.0, lg - lr))
+        fin = np.isfinite(lr)
+        assert np.all(np.isfinite(lg[fin])), f"{what}: non-finite LSE"
+        dl = np.abs(lg[fin] - lr[fin]) if fin.any() else np.zeros(1)
         assert dl.max() <= MAX_ABS_LSE, f"{what}: max|dLSE| = {dl.max():.3e}"
     return float(d.max()), float(d.mean())
 
