@@ -12,10 +12,12 @@ measured HBM bandwidth, and value = 100 * (sum over ranks of ideal time) /
 summed over the GPUs of the job.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                    [--workload step|long]
+                    [--workload step|long|varlen]
 
 `--workload long` times the long-context pair (T=S=16384 prefill and a
-131072-token split-KV decode) with the same accounting.  `--impl reference`
+131072-token split-KV decode) with the same accounting; `--workload varlen`
+replaces the prefill by 16 packed sequences of U[64, 2048] tokens
+(attn_fwd_varlen).  `--impl reference`
 times the fp64 CPU oracle (the only reference implementation there is) on a
 bounded sample of the same step.
 """
@@ -39,7 +41,50 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 WORKLOAD_SETS = {
     "step": ("llama3_8b_prefill", "paged_decode_b64"),
     "long": ("long_prefill_16k", "long_decode_131k"),
+    "varlen": ("varlen_prefill_16seq", "paged_decode_b64"),
 }
+
+
+class PrefillCase:
+    """The prefill half of a step: dense (attn_fwd) or packed (attn_fwd_varlen)."""
+
+    def __init__(self, name, seed, dev, fa, inputs, workloads):
+        import torch
+        self.name = name
+        self.varlen = name in inputs.VARLEN_WORKLOADS
+        if self.varlen:
+            sp = self.spec = inputs.VARLEN_WORKLOADS[name]
+            vin = inputs.make_varlen(sp, seed=seed)
+            self.host_in = [vin.q, vin.k, vin.v, vin.cu_q, vin.cu_k]
+            lens_q = (vin.cu_q[1:] - vin.cu_q[:-1]).tolist()
+            lens_k = (vin.cu_k[1:] - vin.cu_k[:-1]).tolist()
+            self.flops = sum(workloads.prefill_flops(1, sp.Hq, t, s_, sp.d, sp.causal) for t, s_ in zip(lens_q, lens_k))
+            self.max_q, self.total_q, self.total_k = vin.max_q, int(vin.cu_q[-1]), int(vin.cu_k[-1])
+            self.dev_in = [t.to(dev) for t in self.host_in]
+            self.o = torch.empty_like(self.dev_in[0])
+            self.lse = torch.empty(sp.Hq, self.total_q, device=dev, dtype=torch.float32)
+            self.config = {**vars_of(sp), "lengths": lens_q, "total_tokens": self.total_q}
+        else:
+            sp = self.spec = inputs.WORKLOADS[name]
+            q, k, v = inputs.make_prefill(sp, seed=seed)
+            self.host_in = [q, k, v]
+            self.flops = workloads.prefill_flops(sp.B, sp.Hq, sp.T, sp.S, sp.d, sp.causal)
+            self.dev_in = [t.to(dev) for t in self.host_in]
+            self.o = torch.empty_like(self.dev_in[0])
+            self.lse = torch.empty(sp.B, sp.Hq, sp.T, device=dev, dtype=torch.float32)
+            self.config = vars_of(sp)
+        self.fa = fa
+
+    def call(self, stream):
+        sp, fa = self.spec, self.fa
+        if self.varlen:
+            q, k, v, cq, ck = self.dev_in
+            fa.attn_fwd_varlen(q, k, v, self.o, self.lse, cq, ck, sp.B, self.max_q, self.total_q, self.total_k,
+                               sp.Hq, sp.Hkv, sp.d, sp.causal, sp.scale, stream)
+        else:
+            q, k, v = self.dev_in
+            fa.attn_fwd(q, k, v, self.o, self.lse, sp.B, sp.Hq, sp.Hkv, sp.T, sp.S, sp.d, sp.causal, sp.scale,
+                        stream)
 
 
 def load_peaks():
@@ -126,8 +171,41 @@ class ClockSampler:
 # --------------------------------------------------------------------------
 # CPU baseline: the fp64 oracle on a bounded sample of the same step
 # --------------------------------------------------------------------------
+def _cpu_prefill_dense(pname, seed_offset, orc, inputs, workloads, f):
+    """Oracle time of a dense prefill, from an evenly spread set of rows of
+    batch 0 (all heads), scaled by visible pairs to the whole workload."""
+    ps = inputs.WORKLOADS[pname]
+    q, k, v = inputs.make_prefill(ps, seed=ps.seed + seed_offset)
+    qd, kd, vd = f(q), f(k), f(v)
+    T = ps.T
+    rows = list(range(0, T, max(1, T // 64)))
+    t0 = time.perf_counter()
+    orc.attention(qd[:1], kd[:1], vd[:1], ps.scale, ps.causal, rows=rows)
+    tp = time.perf_counter() - t0
+    seen = sum(min(ps.S, i + ps.S - ps.T + 1) if ps.causal else ps.S for i in rows)  # cost ~ keys seen
+    full_pairs = workloads.visible_pairs(ps.T, ps.S, ps.causal) * ps.B
+    flops = workloads.prefill_flops(ps.B, ps.Hq, ps.T, ps.S, ps.d, ps.causal)
+    return tp * full_pairs / max(seen, 1), flops, f"rows {len(rows)}/{T} of batch 0 (all {ps.Hq} heads)"
+
+
+def _cpu_prefill_varlen(pname, seed_offset, orc, inputs, workloads, f):
+    """Oracle time of a packed prefill, from its first two sequences, scaled
+    by visible pairs to all sequences."""
+    sp = inputs.VARLEN_WORKLOADS[pname]
+    vin = inputs.make_varlen(sp, seed=sp.seed + seed_offset)
+    lq = (vin.cu_q[1:] - vin.cu_q[:-1]).tolist()
+    lk = (vin.cu_k[1:] - vin.cu_k[:-1]).tolist()
+    n = 2
+    cq, ck = vin.cu_q[:n + 1].numpy(), vin.cu_k[:n + 1].numpy()
+    t0 = time.perf_counter()
+    orc.attention_varlen(f(vin.q[:cq[-1]]), f(vin.k[:ck[-1]]), f(vin.v[:ck[-1]]), cq, ck, sp.scale, sp.causal)
+    tp = time.perf_counter() - t0
+    pairs = [workloads.visible_pairs(t, s_, sp.causal) for t, s_ in zip(lq, lk)]
+    flops = sum(workloads.prefill_flops(1, sp.Hq, t, s_, sp.d, sp.causal) for t, s_ in zip(lq, lk))
+    return tp * sum(pairs) / max(sum(pairs[:n]), 1), flops, f"sequences {n}/{sp.B} (all {sp.Hq} heads)"
+
+
 def cpu_baseline(pname, dname, peaks, seed_offset=0, budget_s=20.0):
-    import numpy as np
     import torch
 
     from flashattention_attention_attn_b200 import inputs, workloads
@@ -138,22 +216,13 @@ def cpu_baseline(pname, dname, peaks, seed_offset=0, budget_s=20.0):
         cores = max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
     except Exception:
         cores = 1
-    ps = inputs.WORKLOADS[pname]
-    ds = inputs.WORKLOADS[dname]
-    q, k, v = inputs.make_prefill(ps, seed=ps.seed + seed_offset)
-    dinp = inputs.make_paged(ds, seed=ds.seed + seed_offset)
     f = lambda t: t.to(torch.float64).numpy()  # noqa: E731
-    qd, kd, vd = f(q), f(k), f(v)
-    # prefill sample: all heads of batch 0, an evenly spread set of rows
-    T = ps.T
-    rows = list(range(0, T, max(1, T // 64)))
-    t0 = time.perf_counter()
-    orc.attention(qd[:1], kd[:1], vd[:1], ps.scale, ps.causal, rows=rows)
-    tp = time.perf_counter() - t0
-    # cost of a row is proportional to the keys it sees
-    seen = sum(min(ps.S, i + ps.S - ps.T + 1) if ps.causal else ps.S for i in rows)
-    full_pairs = workloads.visible_pairs(ps.T, ps.S, ps.causal) * ps.B
-    t_prefill = tp * full_pairs / max(seen, 1)
+    if pname in inputs.VARLEN_WORKLOADS:
+        t_prefill, flops, pdesc = _cpu_prefill_varlen(pname, seed_offset, orc, inputs, workloads, f)
+    else:
+        t_prefill, flops, pdesc = _cpu_prefill_dense(pname, seed_offset, orc, inputs, workloads, f)
+    ds = inputs.WORKLOADS[dname]
+    dinp = inputs.make_paged(ds, seed=ds.seed + seed_offset)
     # decode sample: leading sequences until ~budget/2 spent or 4 sequences
     lens = dinp.seq_lens.numpy()
     kc, vc = f(dinp.k_cache), f(dinp.v_cache)
@@ -168,14 +237,12 @@ def cpu_baseline(pname, dname, peaks, seed_offset=0, budget_s=20.0):
         if nseq >= 4 or td > budget_s / 2:
             break
     t_decode = td * float(lens.sum()) / max(done_tok, 1)
-    flops = workloads.prefill_flops(ps.B, ps.Hq, ps.T, ps.S, ps.d, ps.causal)
     dbytes = workloads.decode_bytes(lens, ds.Hq, ds.Hkv, ds.d, ds.block_size)
     ideal = flops / (peaks["bf16_tflops"] * 1e12) + dbytes / (peaks["hbm_gbs"] * 1e9)
     est = t_prefill + t_decode
     return {"value": 100.0 * ideal / est, "unit": UNIT, "cores": int(cores), "kind": "oracle",
-            "sample": (f"fp64 oracle: prefill rows {len(rows)}/{T} of batch 0 (all {ps.Hq} heads), "
-                       f"decode {nseq}/{len(lens)} sequences ({done_tok} tokens); time scaled by visible "
-                       f"pairs / tokens to the full step"),
+            "sample": (f"fp64 oracle: prefill {pdesc}, decode {nseq}/{len(lens)} sequences ({done_tok} tokens); "
+                       f"time scaled by visible pairs / tokens to the full step"),
             "est_step_s": est}
 
 
@@ -210,26 +277,23 @@ def main():
     if fa.attn_check_support(local_rank) != 0:
         raise RuntimeError("device not supported by the library")
 
-    ps = inputs.WORKLOADS[pname]
     ds = inputs.WORKLOADS[dname]
     # weak scaling: every rank runs its own batch (different seeds), no exchange
-    q, k, v = inputs.make_prefill(ps, seed=dist_util.rank_seed(ps.seed, rank))
+    pspec = inputs.VARLEN_WORKLOADS.get(pname) or inputs.WORKLOADS[pname]
+    pre = PrefillCase(pname, dist_util.rank_seed(pspec.seed, rank), dev, fa, inputs, workloads)
     dinp = inputs.make_paged(ds, seed=dist_util.rank_seed(ds.seed, rank))
-    dq, dk, dv = q.to(dev), k.to(dev), v.to(dev)
-    o = torch.empty_like(dq)
-    lse = torch.empty(ps.B, ps.Hq, ps.T, device=dev, dtype=torch.float32)
     qd_, kc, vc = dinp.q.to(dev), dinp.k_cache.to(dev), dinp.v_cache.to(dev)
     bt, sl = dinp.block_table.to(dev), dinp.seq_lens.to(dev)
     od = torch.empty(ds.B, ds.Hq, ds.d, device=dev, dtype=torch.bfloat16)
     maxb = dinp.block_table.shape[1]
     stream = torch.cuda.current_stream(dev)
 
-    flops = workloads.prefill_flops(ps.B, ps.Hq, ps.T, ps.S, ps.d, ps.causal)
+    flops = pre.flops
     dbytes = workloads.decode_bytes(dinp.seq_lens.tolist(), ds.Hq, ds.Hkv, ds.d, ds.block_size)
     splits = args.num_splits
 
     def step():
-        fa.attn_fwd(dq, dk, dv, o, lse, ps.B, ps.Hq, ps.Hkv, ps.T, ps.S, ps.d, ps.causal, ps.scale, stream)
+        pre.call(stream)
         fa.paged_attn_decode(qd_, kc, vc, bt, sl, ds.B, ds.Hq, ds.Hkv, ds.d, ds.block_size, maxb, splits, od,
                              stream)
 
@@ -251,7 +315,7 @@ def main():
     start.record(stream)
     for i in range(K):
         ev[i][0].record(stream)
-        fa.attn_fwd(dq, dk, dv, o, lse, ps.B, ps.Hq, ps.Hkv, ps.T, ps.S, ps.d, ps.causal, ps.scale, stream)
+        pre.call(stream)
         ev[i][1].record(stream)
         fa.paged_attn_decode(qd_, kc, vc, bt, sl, ds.B, ds.Hq, ds.Hkv, ds.d, ds.block_size, maxb, splits, od,
                              stream)
@@ -281,11 +345,11 @@ def main():
     e2e = None
     if args.e2e_steps > 0:
         pin = lambda t: t.pin_memory()  # noqa: E731
-        h_in = [pin(q), pin(k), pin(v), pin(dinp.q), pin(dinp.k_cache), pin(dinp.v_cache),
-                pin(dinp.block_table), pin(dinp.seq_lens)]
-        d_in = [dq, dk, dv, qd_, kc, vc, bt, sl]
-        h_o = torch.empty(o.shape, dtype=o.dtype).pin_memory()
-        h_lse = torch.empty(lse.shape, dtype=lse.dtype).pin_memory()
+        h_in = [pin(t) for t in pre.host_in] + [pin(dinp.q), pin(dinp.k_cache), pin(dinp.v_cache),
+                                                pin(dinp.block_table), pin(dinp.seq_lens)]
+        d_in = list(pre.dev_in) + [qd_, kc, vc, bt, sl]
+        h_o = torch.empty(pre.o.shape, dtype=pre.o.dtype).pin_memory()
+        h_lse = torch.empty(pre.lse.shape, dtype=pre.lse.dtype).pin_memory()
         h_od = torch.empty(od.shape, dtype=od.dtype).pin_memory()
         h2d = sum(t.numel() * t.element_size() for t in h_in)
         d2h = sum(t.numel() * t.element_size() for t in (h_o, h_lse, h_od))
@@ -299,8 +363,8 @@ def main():
             for h, d_ in zip(h_in, d_in):
                 d_.copy_(h, non_blocking=True)
             step()
-            h_o.copy_(o, non_blocking=True)
-            h_lse.copy_(lse, non_blocking=True)
+            h_o.copy_(pre.o, non_blocking=True)
+            h_lse.copy_(pre.lse, non_blocking=True)
             h_od.copy_(od, non_blocking=True)
         e1.record(stream)
         torch.cuda.synchronize()
@@ -332,7 +396,7 @@ def main():
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K, "warmup": args.warmup,
         "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "bf16", "data": "synthetic (seeded N(0,1) bf16; random block-id permutations)",
-        "config": {"workload": f"{pname} + {dname}", "prefill": vars_of(ps), "decode": vars_of(ds),
+        "config": {"workload": f"{pname} + {dname}", "prefill": pre.config, "decode": vars_of(ds),
                    "decode_num_splits": splits or "auto", "parallelism": f"replicas x{world} (no exchange)",
                    "l2": "inputs larger than L2 (decode KV cache %.0f MB per step)" % (dbytes / 1e6)},
         "parts": {"prefill": {"ms": t_pre, "tflops": pre_tflops, "frac": pre_tflops / peaks["bf16_tflops"],
@@ -374,7 +438,7 @@ def run_reference(args, pname, dname, peaks, peak_src, world):
         "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": est * 1e3, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic (same seeds as ours)",
-        "config": {"workload": f"{pname} + {dname}", "prefill": vars_of(inputs.WORKLOADS[pname]),
+        "config": {"workload": f"{pname} + {dname}", "prefill": vars_of(inputs.VARLEN_WORKLOADS.get(pname) or inputs.WORKLOADS[pname]),
                    "decode": vars_of(inputs.WORKLOADS[dname])},
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": info["cores"], "kind": "oracle",
                          "sample": info["sample"]},

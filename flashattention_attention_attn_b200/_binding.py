@@ -37,6 +37,9 @@ def library() -> ctypes.CDLL:
         c_int, c_float, vp = ctypes.c_int, ctypes.c_float, ctypes.c_void_p
         lib.attn_fwd.argtypes = [vp, vp, vp, vp, vp, c_int, c_int, c_int, c_int, c_int, c_int, c_int, c_float, vp]
         lib.attn_fwd.restype = c_int
+        lib.attn_fwd_varlen.argtypes = [vp, vp, vp, vp, vp, vp, vp, c_int, c_int, c_int, c_int, c_int, c_int, c_int,
+                                        c_int, c_float, vp]
+        lib.attn_fwd_varlen.restype = c_int
         lib.paged_attn_decode.argtypes = [vp, vp, vp, vp, vp, c_int, c_int, c_int, c_int, c_int, c_int, c_int,
                                           vp, vp]
         lib.paged_attn_decode.restype = c_int
@@ -83,6 +86,17 @@ def attn_fwd(q, k, v, o, lse, B, Hq, Hkv, T, S, d, causal, scale, stream=None) -
                             int(S), int(d), int(bool(causal)), float(scale), _stream(stream))
     if rc != ATTN_OK:
         raise AttnError(rc, "attn_fwd")
+
+
+def attn_fwd_varlen(q, k, v, o, lse, cu_seqlens_q, cu_seqlens_k, B, max_seqlen_q, total_q, total_k, Hq, Hkv, d,
+                    causal, scale, stream=None) -> None:
+    """attn_fwd over packed sequences: q [total_q,Hq,d], k/v [total_k,Hkv,d],
+    o [total_q,Hq,d], lse [Hq,total_q] or None, cu_seqlens_* int32 [B+1]."""
+    rc = library().attn_fwd_varlen(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(cu_seqlens_q),
+                                   _ptr(cu_seqlens_k), int(B), int(max_seqlen_q), int(total_q), int(total_k),
+                                   int(Hq), int(Hkv), int(d), int(bool(causal)), float(scale), _stream(stream))
+    if rc != ATTN_OK:
+        raise AttnError(rc, "attn_fwd_varlen")
 
 
 def paged_attn_decode(q, k_cache, v_cache, block_table, seq_lens, B, Hq, Hkv, d, block_size, max_blocks,

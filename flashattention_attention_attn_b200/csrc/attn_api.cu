@@ -69,7 +69,7 @@ int probe_device(int dev, DeviceState** out) {
       st.status = ATTN_ERR_UNSUPPORTED;
     } else {
       cudaFuncAttributes fa;
-      if (cudaFuncGetAttributes(&fa, prefill::prefill_fwd_sm100<128>) != cudaSuccess) {
+      if (cudaFuncGetAttributes(&fa, prefill::prefill_fwd_sm100<128, false>) != cudaSuccess) {
         cudaGetLastError();
         st.status = ATTN_ERR_UNSUPPORTED;  // no sm_100a image for this device
       } else if (encode_tiled() == nullptr) {
@@ -93,8 +93,10 @@ int prepare_device(int dev, DeviceState* st) {
     const void* fn;
     size_t bytes;
   } kernels[] = {
-      {reinterpret_cast<const void*>(prefill::prefill_fwd_sm100<64>), prefill::smem_bytes<64>()},
-      {reinterpret_cast<const void*>(prefill::prefill_fwd_sm100<128>), prefill::smem_bytes<128>()},
+      {reinterpret_cast<const void*>(prefill::prefill_fwd_sm100<64, false>), prefill::smem_bytes<64>()},
+      {reinterpret_cast<const void*>(prefill::prefill_fwd_sm100<128, false>), prefill::smem_bytes<128>()},
+      {reinterpret_cast<const void*>(prefill::prefill_fwd_sm100<64, true>), prefill::smem_bytes<64>()},
+      {reinterpret_cast<const void*>(prefill::prefill_fwd_sm100<128, true>), prefill::smem_bytes<128>()},
       {reinterpret_cast<const void*>(decode::paged_decode_split<64>), decode::smem_bytes<64>()},
       {reinterpret_cast<const void*>(decode::paged_decode_split<128>), decode::smem_bytes<128>()},
   };
@@ -173,7 +175,9 @@ int launch_prefill(const void* q, const void* k, const void* v, void* o, float* 
       make_map_bthd(&mv, v, B, S, Hkv, D) || make_map_bthd(&mo, o, B, T, Hq, D))
     return ATTN_ERR_CUDA;
   prefill::Params p;
+  std::memset(&p, 0, sizeof(p));
   p.lse = lse;
+  p.o = static_cast<__nv_bfloat16*>(o);
   p.B = B;
   p.Hq = Hq;
   p.Hkv = Hkv;
@@ -184,8 +188,41 @@ int launch_prefill(const void* q, const void* k, const void* v, void* o, float* 
   p.num_mblocks = (T + 2 * prefill::kBM - 1) / (2 * prefill::kBM);
   const long long grid = static_cast<long long>(p.num_mblocks) * Hq * B;
   if (grid > 0x7fffffffLL) return ATTN_ERR_UNSUPPORTED;
-  prefill::prefill_fwd_sm100<D><<<static_cast<unsigned>(grid), prefill::kThreads, prefill::smem_bytes<D>(),
-                                  stream>>>(mq, mk, mv, mo, p);
+  prefill::prefill_fwd_sm100<D, false><<<static_cast<unsigned>(grid), prefill::kThreads,
+                                         prefill::smem_bytes<D>(), stream>>>(mq, mk, mv, mo, p);
+  return launch_status();
+}
+
+// Packed sequences: the maps see [total, H, D] as one batch; the grid covers
+// ceil(max_seqlen_q / 256) query blocks of every (sequence, head) and CTAs
+// past a sequence's end exit at once.
+template <int D>
+int launch_prefill_varlen(const void* q, const void* k, const void* v, void* o, float* lse, const int32_t* cu_q,
+                          const int32_t* cu_k, int B, int max_q, int total_q, int total_k, int Hq, int Hkv,
+                          int causal, float scale, cudaStream_t stream) {
+  CUtensorMap mq, mk, mv, mo;
+  if (make_map_bthd(&mq, q, 1, total_q, Hq, D) || make_map_bthd(&mk, k, 1, total_k, Hkv, D) ||
+      make_map_bthd(&mv, v, 1, total_k, Hkv, D) || make_map_bthd(&mo, o, 1, total_q, Hq, D))
+    return ATTN_ERR_CUDA;
+  prefill::Params p;
+  std::memset(&p, 0, sizeof(p));
+  p.lse = lse;
+  p.o = static_cast<__nv_bfloat16*>(o);
+  p.cu_q = cu_q;
+  p.cu_k = cu_k;
+  p.B = B;
+  p.Hq = Hq;
+  p.Hkv = Hkv;
+  p.T = max_q;
+  p.S = 0;
+  p.total_q = total_q;
+  p.causal = causal ? 1 : 0;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  p.num_mblocks = (max_q + 2 * prefill::kBM - 1) / (2 * prefill::kBM);
+  const long long grid = static_cast<long long>(p.num_mblocks) * Hq * B;
+  if (grid > 0x7fffffffLL) return ATTN_ERR_UNSUPPORTED;
+  prefill::prefill_fwd_sm100<D, true><<<static_cast<unsigned>(grid), prefill::kThreads,
+                                        prefill::smem_bytes<D>(), stream>>>(mq, mk, mv, mo, p);
   return launch_status();
 }
 
@@ -327,6 +364,39 @@ extern "C" int attn_fwd(const void* q, const void* k, const void* v, void* o, fl
   }
   if (d == 64) return launch_prefill<64>(q, k, v, o, lse, B, Hq, Hkv, T, S, causal, scale, stream);
   return launch_prefill<128>(q, k, v, o, lse, B, Hq, Hkv, T, S, causal, scale, stream);
+}
+
+extern "C" int attn_fwd_varlen(const void* q, const void* k, const void* v, void* o, float* lse,
+                               const int32_t* cu_seqlens_q, const int32_t* cu_seqlens_k, int B, int max_seqlen_q,
+                               int total_q, int total_k, int Hq, int Hkv, int d, int causal, float scale,
+                               attn_stream_t stream_) {
+  cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+  if (B < 0 || max_seqlen_q < 0 || total_q < 0 || total_k < 0 || Hq <= 0 || Hkv <= 0 || d <= 0)
+    return ATTN_ERR_INVALID_ARG;
+  if (Hq % Hkv != 0) return ATTN_ERR_INVALID_ARG;
+  if (!(scale > 0.f) || !std::isfinite(scale)) return ATTN_ERR_INVALID_ARG;
+  if (B == 0 || total_q == 0 || max_seqlen_q == 0) return ATTN_OK;
+  if (q == nullptr || o == nullptr || cu_seqlens_q == nullptr || cu_seqlens_k == nullptr) return ATTN_ERR_INVALID_ARG;
+  if (total_k > 0 && (k == nullptr || v == nullptr)) return ATTN_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return ATTN_ERR_UNSUPPORTED;
+  if (!aligned16(q) || !aligned16(o) || (total_k > 0 && (!aligned16(k) || !aligned16(v)))) return ATTN_ERR_UNSUPPORTED;
+  if ((lse != nullptr && (reinterpret_cast<uintptr_t>(lse) & 3u)) ||
+      (reinterpret_cast<uintptr_t>(cu_seqlens_q) & 3u) || (reinterpret_cast<uintptr_t>(cu_seqlens_k) & 3u))
+    return ATTN_ERR_UNSUPPORTED;
+  DeviceState* st = nullptr;
+  int rc = current_device_state(&st);
+  if (rc != ATTN_OK) return rc;
+  if (total_k == 0) {  // no key anywhere: O = 0, LSE = -inf
+    const size_t n_o = static_cast<size_t>(total_q) * Hq * d;
+    const size_t n_lse = static_cast<size_t>(Hq) * total_q;
+    fill_no_keys<<<st->sms * 4, 256, 0, stream>>>(static_cast<__nv_bfloat16*>(o), lse, n_o, n_lse);
+    return launch_status();
+  }
+  if (d == 64)
+    return launch_prefill_varlen<64>(q, k, v, o, lse, cu_seqlens_q, cu_seqlens_k, B, max_seqlen_q, total_q, total_k,
+                                     Hq, Hkv, causal, scale, stream);
+  return launch_prefill_varlen<128>(q, k, v, o, lse, cu_seqlens_q, cu_seqlens_k, B, max_seqlen_q, total_q, total_k,
+                                    Hq, Hkv, causal, scale, stream);
 }
 
 extern "C" int paged_attn_decode(const void* q, const void* k_cache, const void* v_cache,

@@ -123,8 +123,12 @@ constexpr size_t smem_bytes() {
 }
 
 struct Params {
-  float* lse;  // [B, Hq, T] or nullptr
-  int B, Hq, Hkv, T, S;
+  float* lse;             // [B, Hq, T] (dense) / [Hq, total_q] (varlen), or nullptr
+  __nv_bfloat16* o;       // output base (row stores of ragged varlen tiles)
+  const int32_t* cu_q;    // varlen: [B + 1] prefix sums of query lengths
+  const int32_t* cu_k;    // varlen: [B + 1] prefix sums of key lengths
+  int B, Hq, Hkv, T, S;   // dense: T, S; varlen: T = max query length
+  int total_q;            // varlen: rows of the packed query tensor
   int causal;
   float scale_log2;  // scale * log2(e)
   int num_mblocks;   // ceil(T / 256)
@@ -132,16 +136,19 @@ struct Params {
 
 // Keys visible to the query tile with rows [r0, r0 + 128) (ragged T clipped)
 // as a number of kBN-wide K/V tiles; 0 when no row of it sees any key.
-__device__ __forceinline__ int kv_tiles_for(int r0, const Params& p) {
-  if (r0 >= p.T) return 0;
-  const int r1 = min(r0 + kBM, p.T);
-  int kmax = p.S - 1;
-  if (p.causal) kmax = min(kmax, r1 - 1 + (p.S - p.T));
+__device__ __forceinline__ int kv_tiles_for(int r0, int T, int S, int causal) {
+  if (r0 >= T) return 0;
+  const int r1 = min(r0 + kBM, T);
+  int kmax = S - 1;
+  if (causal) kmax = min(kmax, r1 - 1 + (S - T));
   if (kmax < 0) return 0;
   return kmax / kBN + 1;
 }
 
-template <int D>
+// VARLEN: packed sequences (no padding).  The tensor maps then cover
+// [total, H, D] as batch 1, and each CTA takes its sequence's row offsets
+// and lengths from cu_q / cu_k.
+template <int D, bool VARLEN>
 __global__ void __launch_bounds__(kThreads, 1)
     prefill_fwd_sm100(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                       const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
@@ -162,8 +169,17 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int b = rem / p.Hq;
   const int hk = h / (p.Hq / p.Hkv);
   const int m0 = mb * 2 * kBM;
-  const int n0 = kv_tiles_for(m0, p);
-  const int n1 = kv_tiles_for(m0 + kBM, p);
+  int T = p.T, S = p.S, qoff = 0, koff = 0, bc = b;  // bc: batch coordinate of the maps
+  if constexpr (VARLEN) {
+    qoff = p.cu_q[b];
+    T = p.cu_q[b + 1] - qoff;
+    koff = p.cu_k[b];
+    S = p.cu_k[b + 1] - koff;
+    bc = 0;
+    if (m0 >= T) return;  // this query block lies past the sequence (uniform over the CTA)
+  }
+  const int n0 = kv_tiles_for(m0, T, S, p.causal);
+  const int n1 = kv_tiles_for(m0 + kBM, T, S, p.causal);
   const int n_max = max(n0, n1);
 
   if (threadIdx.x == 0) {
@@ -204,7 +220,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (nt[t] == 0) continue;
         mbar_arrive_expect_tx(&sm.q_full[t], C::kTileBytes);
         for (int c = 0; c < C::kChunks; ++c)
-          tma_load_4d(sm.q[t][c], &tmQ, &sm.q_full[t], c * 64, h, m0 + t * kBM, b);
+          tma_load_4d(sm.q[t][c], &tmQ, &sm.q_full[t], c * 64, h, qoff + m0 + t * kBM, bc);
       }
       int k_issued = 0, v_issued = 0;  // K / V tiles whose loads were issued
       for (int j = 0; j < n_max; ++j) {
@@ -213,12 +229,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!mbar_wait(&sm.k_empty[s], ph ^ 1, abort_flag)) break;
         mbar_arrive_expect_tx(&sm.k_full[s], C::kTileBytes);
         for (int c = 0; c < C::kChunks; ++c)
-          tma_load_4d(sm.k[s][c], &tmK, &sm.k_full[s], c * 64, hk, j * kBN, b);
+          tma_load_4d(sm.k[s][c], &tmK, &sm.k_full[s], c * 64, hk, koff + j * kBN, bc);
         k_issued = j + 1;
         if (!mbar_wait(&sm.v_empty[s], ph ^ 1, abort_flag)) break;
         mbar_arrive_expect_tx(&sm.v_full[s], C::kTileBytes);
         for (int c = 0; c < C::kChunks; ++c)
-          tma_load_4d(sm.v[s][c], &tmV, &sm.v_full[s], c * 64, hk, j * kBN, b);
+          tma_load_4d(sm.v[s][c], &tmV, &sm.v_full[s], c * 64, hk, koff + j * kBN, bc);
         v_issued = j + 1;
       }
       if (*abort_flag) {
@@ -311,7 +327,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t lane_off = uint32_t((warp & 3) * 32) << 16;
     const uint32_t tS = tmem + lane_off + t * kBN;
     const uint32_t tO = tmem + lane_off + 2 * kBN + t * D;
-    const int visible = p.causal ? min(p.S, row + (p.S - p.T) + 1) : p.S;
+    const int visible = p.causal ? min(S, row + (S - T) + 1) : S;
     const float sl2 = p.scale_log2;
 
     float m_used = -INFINITY;  // reference max, log2 domain
@@ -427,14 +443,27 @@ __global__ void __launch_bounds__(kThreads, 1)
             make_uint4(pk[4 * q4], pk[4 * q4 + 1], pk[4 * q4 + 2], pk[4 * q4 + 3]);
       }
     }
-    if (p.lse != nullptr && row < p.T) {
+    if (p.lse != nullptr && row < T) {
       const float lse = (l > 0.f) ? (m_used + __log2f(l)) * 0.69314718055994531f : -INFINITY;
-      p.lse[(static_cast<size_t>(b) * p.Hq + h) * p.T + row] = lse;
+      const size_t lse_rows = VARLEN ? static_cast<size_t>(p.total_q) : static_cast<size_t>(T);
+      p.lse[(static_cast<size_t>(bc) * p.Hq + h) * lse_rows + qoff + row] = lse;
     }
     fence_proxy_async_smem();
     named_barrier_sync(1 + t, kBM);
-    if (r == 0 && m0 + t * kBM < p.T) {
-      for (int c = 0; c < C::kChunks; ++c) tma_store_4d(&tmO, stage + c * C::kChunkBytes, c * 64, h, m0 + t * kBM, b);
+    const int r0 = m0 + t * kBM;
+    if (VARLEN && r0 + kBM > T) {
+      // The tile crosses the end of the sequence: a 128-row store would
+      // overwrite the next sequence's rows, so each thread stores its own row.
+      if (row < T) {
+        uint8_t* dst = reinterpret_cast<uint8_t*>(p.o) + ((static_cast<size_t>(qoff) + row) * p.Hq + h) * D * 2;
+#pragma unroll
+        for (int u = 0; u < D / 8; ++u) {
+          const uint8_t* src = stage + (u / 8) * C::kChunkBytes + r * 128 + (((u & 7) ^ (r & 7)) << 4);
+          *reinterpret_cast<uint4*>(dst + u * 16) = *reinterpret_cast<const uint4*>(src);
+        }
+      }
+    } else if (r == 0 && r0 < T) {
+      for (int c = 0; c < C::kChunks; ++c) tma_store_4d(&tmO, stage + c * C::kChunkBytes, c * 64, h, qoff + r0, bc);
       tma_store_commit();
       tma_store_wait_read0();
     }

@@ -74,6 +74,28 @@ WORKLOADS = {
 }
 
 
+@dataclass(frozen=True)
+class VarlenSpec:
+    B: int
+    Hq: int
+    Hkv: int
+    d: int
+    len_lo: int
+    len_hi: int
+    causal: bool = True
+    seed: int = 0
+
+    @property
+    def scale(self) -> float:
+        return 1.0 / (self.d ** 0.5)
+
+
+# 16 packed Llama3-8B-shaped sequences, lengths uniform in [64, 2048]
+VARLEN_WORKLOADS = {
+    "varlen_prefill_16seq": VarlenSpec(B=16, Hq=32, Hkv=8, d=128, len_lo=64, len_hi=2048, causal=True, seed=1005),
+}
+
+
 def _randn_bf16(gen: torch.Generator, shape) -> torch.Tensor:
     return torch.randn(*shape, generator=gen, dtype=torch.float32).to(BF16)
 
@@ -166,3 +188,37 @@ def permute_pool(inp: PagedInputs, seed: int) -> PagedInputs:
     table[used] = perm[table[used].long()].to(torch.int32)
     return PagedInputs(q=inp.q, k_cache=k2, v_cache=v2, block_table=table,
                        seq_lens=inp.seq_lens, block_size=inp.block_size)
+
+
+@dataclass
+class VarlenInputs:
+    q: torch.Tensor      # [total_q, Hq, d] bf16
+    k: torch.Tensor      # [total_k, Hkv, d] bf16
+    v: torch.Tensor      # [total_k, Hkv, d] bf16
+    cu_q: torch.Tensor   # [B + 1] int32
+    cu_k: torch.Tensor   # [B + 1] int32
+
+    @property
+    def max_q(self) -> int:
+        return int((self.cu_q[1:] - self.cu_q[:-1]).max()) if self.cu_q.numel() > 1 else 0
+
+
+def make_varlen(spec: VarlenSpec, q_lens=None, k_lens=None, seed: int | None = None) -> VarlenInputs:
+    """Packed sequences.  Draw order: query lengths (uniform in
+    [len_lo, len_hi] unless given), then q, k, v.  Key lengths equal the
+    query lengths (self-attention prefill) unless `k_lens` is given."""
+    s = spec
+    gen = torch.Generator(device="cpu").manual_seed(s.seed if seed is None else seed)
+    if q_lens is None:
+        q_lens = torch.randint(s.len_lo, s.len_hi + 1, (s.B,), generator=gen, dtype=torch.int64).tolist()
+    q_lens = [int(x) for x in q_lens]
+    k_lens = list(q_lens) if k_lens is None else [int(x) for x in k_lens]
+    assert len(q_lens) == len(k_lens) == s.B
+    cu_q = torch.zeros(s.B + 1, dtype=torch.int32)
+    cu_k = torch.zeros(s.B + 1, dtype=torch.int32)
+    cu_q[1:] = torch.cumsum(torch.tensor(q_lens, dtype=torch.int64), 0).to(torch.int32)
+    cu_k[1:] = torch.cumsum(torch.tensor(k_lens, dtype=torch.int64), 0).to(torch.int32)
+    q = _randn_bf16(gen, (int(cu_q[-1]), s.Hq, s.d))
+    k = _randn_bf16(gen, (int(cu_k[-1]), s.Hkv, s.d))
+    v = _randn_bf16(gen, (int(cu_k[-1]), s.Hkv, s.d))
+    return VarlenInputs(q=q, k=k, v=v, cu_q=cu_q, cu_k=cu_k)

@@ -82,6 +82,34 @@ int attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
              attn_stream_t stream);
 
 /*
+ * attn_fwd_varlen - attn_fwd over packed sequences of different lengths,
+ * with no padding (the "dynamic sequence lengths without padding" of the
+ * FlashAttention-2 item on the page "内核更新内容一览", section 关键技术点).
+ *
+ *   q    [total_q, Hq,  d] bf16   the B sequences' queries, back to back
+ *   k    [total_k, Hkv, d] bf16   their keys, back to back
+ *   v    [total_k, Hkv, d] bf16
+ *   o    [total_q, Hq,  d] bf16   (written)
+ *   lse  [Hq, total_q]     fp32   (written; may be NULL)
+ *   cu_seqlens_q, cu_seqlens_k: device int32 [B + 1] prefix sums: sequence b
+ *   owns query rows [cu_seqlens_q[b], cu_seqlens_q[b+1]) and key rows
+ *   [cu_seqlens_k[b], cu_seqlens_k[b+1]); cu_seqlens_*[0] = 0 and
+ *   cu_seqlens_*[B] = total_*.  Lengths may differ between q and k and may
+ *   be 0.  max_seqlen_q must be >= every query length (rows beyond it are
+ *   not computed).
+ *
+ *   Each sequence is attended on its own with the rules of attn_fwd
+ *   (bottom-right causal alignment per sequence with its own T and S, GQA
+ *   map, O = 0 / LSE = -inf for rows that see no key).  Keys of other
+ *   sequences are never given weight; inputs are assumed finite.
+ *   Supported and errors: as attn_fwd; B == 0 or total_q == 0 is a no-op.
+ */
+int attn_fwd_varlen(const void* q, const void* k, const void* v, void* o, float* lse,
+                    const int32_t* cu_seqlens_q, const int32_t* cu_seqlens_k,
+                    int B, int max_seqlen_q, int total_q, int total_k,
+                    int Hq, int Hkv, int d, int causal, float scale, attn_stream_t stream);
+
+/*
  * paged_attn_decode - one query token per sequence against a paged KV cache.
  *
  *   q            [B, Hq, d]                         bf16

@@ -1,6 +1,7 @@
 """fp64 CPU oracle (test infrastructure; never used by the product path)."""
 from .fp64_attention import (  # noqa: F401
     attention,
+    attention_varlen,
     gather_paged_kv,
     paged_decode,
     softmax_rows,

@@ -49,6 +49,7 @@ __all__ = [
     "visible_key_count",
     "softmax_rows",
     "attention",
+    "attention_varlen",
     "gather_paged_kv",
     "paged_decode",
     "split_paged_decode",
@@ -127,6 +128,30 @@ def attention(q, k, v, scale: float, causal: bool, rows=None):
                 O[b, ids, h, :] = P @ Vh
                 with np.errstate(divide="ignore"):
                     LSE[b, h, ids] = np.where(l > 0, m + np.log(np.where(l > 0, l, 1.0)), -np.inf)
+    return O, LSE
+
+
+def attention_varlen(q, k, v, cu_q, cu_k, scale: float, causal: bool):
+    """Packed sequences without padding ("dynamic sequence lengths without
+    padding", FlashAttention-2 item of "内核更新内容一览", section 关键技术点).
+
+    q: [total_q, Hq, d]; k, v: [total_k, Hkv, d]; cu_q, cu_k: [B + 1] prefix
+    sums.  Sequence b is attended on its own (rows cu_q[b]..cu_q[b+1] against
+    keys cu_k[b]..cu_k[b+1]) with `attention`.  Returns O [total_q, Hq, d]
+    and LSE [Hq, total_q].
+    """
+    q = np.asarray(q, dtype=np.float64)
+    total_q, Hq, d = q.shape
+    O = np.zeros((total_q, Hq, d))
+    LSE = np.full((Hq, total_q), -np.inf)
+    for b in range(len(cu_q) - 1):
+        q0, q1 = int(cu_q[b]), int(cu_q[b + 1])
+        k0, k1 = int(cu_k[b]), int(cu_k[b + 1])
+        if q1 == q0:
+            continue
+        ob, lb = attention(q[None, q0:q1], np.asarray(k)[None, k0:k1], np.asarray(v)[None, k0:k1], scale, causal)
+        O[q0:q1] = ob[0]
+        LSE[:, q0:q1] = lb[0]
     return O, LSE
 
 

@@ -72,3 +72,22 @@ def oracle_decode(inp):
     d = inp.q.shape[-1]
     return orc.paged_decode(f64(inp.q), f64(inp.k_cache), f64(inp.v_cache), inp.block_table.numpy(),
                             inp.seq_lens.numpy(), inp.block_size, 1.0 / np.sqrt(d))
+
+
+def run_varlen(inp, causal, scale, max_q=None):
+    import flashattention_attention_attn_b200 as fa
+    total_q, Hq, d = inp.q.shape
+    total_k, Hkv = inp.k.shape[0], inp.k.shape[1]
+    B = inp.cu_q.numel() - 1
+    dq, dk, dv = inp.q.cuda(), inp.k.cuda(), inp.v.cuda()
+    o = torch.full_like(dq, float("nan"))
+    lse = torch.full((Hq, total_q), float("nan"), device="cuda", dtype=torch.float32)
+    fa.attn_fwd_varlen(dq, dk, dv, o, lse, inp.cu_q.cuda(), inp.cu_k.cuda(), B,
+                       inp.max_q if max_q is None else max_q, total_q, total_k, Hq, Hkv, d, causal, scale)
+    torch.cuda.synchronize()
+    assert fa.attn_read_device_status(clear=True) == 0
+    return o.cpu(), lse.cpu()
+
+
+def oracle_varlen(inp, causal, scale):
+    return orc.attention_varlen(f64(inp.q), f64(inp.k), f64(inp.v), inp.cu_q.numpy(), inp.cu_k.numpy(), scale, causal)

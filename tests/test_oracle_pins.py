@@ -270,3 +270,45 @@ def test_unused_table_entries_are_never_read():
     O2, L2 = orc.paged_decode(q, kc, vc, t2, lens, bs, 0.3)
     np.testing.assert_array_equal(O1, O2)
     np.testing.assert_array_equal(L1, L2)
+
+
+def _varlen_case(seed, q_lens, k_lens, Hq=4, Hkv=2, d=8):
+    rng = np.random.default_rng(seed)
+    cu_q = np.concatenate([[0], np.cumsum(q_lens)]).astype(np.int64)
+    cu_k = np.concatenate([[0], np.cumsum(k_lens)]).astype(np.int64)
+    q = rng.standard_normal((cu_q[-1], Hq, d))
+    k = rng.standard_normal((cu_k[-1], Hkv, d))
+    v = rng.standard_normal((cu_k[-1], Hkv, d))
+    return q, k, v, cu_q, cu_k
+
+
+@pytest.mark.parametrize("causal", [True, False])
+def test_varlen_brute_force_ragged(causal):
+    q_lens, k_lens = [3, 0, 5, 1, 4], [3, 2, 7, 1, 2]
+    q, k, v, cu_q, cu_k = _varlen_case(40, q_lens, k_lens)
+    O, L = orc.attention_varlen(q, k, v, cu_q, cu_k, 0.3, causal)
+    for b in range(len(q_lens)):
+        q0, q1, k0, k1 = cu_q[b], cu_q[b + 1], cu_k[b], cu_k[b + 1]
+        Ob, Lb = _brute_force(q[None, q0:q1], k[None, k0:k1], v[None, k0:k1], 0.3, causal)
+        np.testing.assert_allclose(O[q0:q1], Ob[0], rtol=0, atol=1e-12)
+        np.testing.assert_allclose(L[:, q0:q1], Lb[0], rtol=0, atol=1e-12)
+
+
+def test_varlen_equal_lengths_equal_dense_batch():
+    B, T = 3, 11
+    q, k, v, cu_q, cu_k = _varlen_case(41, [T] * B, [T] * B)
+    O, L = orc.attention_varlen(q, k, v, cu_q, cu_k, 0.3, True)
+    Od, Ld = orc.attention(q.reshape(B, T, 4, 8), k.reshape(B, T, 2, 8), v.reshape(B, T, 2, 8), 0.3, True)
+    np.testing.assert_array_equal(O, Od.reshape(B * T, 4, 8))
+    np.testing.assert_array_equal(L, Ld.transpose(1, 0, 2).reshape(4, B * T))
+
+
+def test_varlen_sequences_do_not_see_each_other():
+    q, k, v, cu_q, cu_k = _varlen_case(42, [4, 6, 3], [5, 6, 2])
+    O1, L1 = orc.attention_varlen(q, k, v, cu_q, cu_k, 0.3, True)
+    k2, v2 = k.copy(), v.copy()
+    k2[cu_k[1]:] = 100.0  # rewrite the keys/values of sequences 1 and 2
+    v2[cu_k[1]:] = -7.0
+    O2, L2 = orc.attention_varlen(q, k2, v2, cu_q, cu_k, 0.3, True)
+    np.testing.assert_array_equal(O1[:cu_q[1]], O2[:cu_q[1]])
+    np.testing.assert_array_equal(L1[:, :cu_q[1]], L2[:, :cu_q[1]])
