@@ -12,12 +12,13 @@ measured HBM bandwidth, and value = 100 * (sum over ranks of ideal time) /
 summed over the GPUs of the job.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                    [--workload step|long|varlen]
+                    [--workload step|long|varlen|chunked]
 
 `--workload long` times the long-context pair (T=S=16384 prefill and a
 131072-token split-KV decode) with the same accounting; `--workload varlen`
 replaces the prefill by 16 packed sequences of U[64, 2048] tokens
-(attn_fwd_varlen).  `--impl reference`
+(attn_fwd_varlen); `--workload chunked` by a 512-token chunk of each of 8
+sequences against their paged cache of 1k-8k tokens (paged_attn_prefill).  `--impl reference`
 times the fp64 CPU oracle (the only reference implementation there is) on a
 bounded sample of the same step.
 """
@@ -42,17 +43,33 @@ WORKLOAD_SETS = {
     "step": ("llama3_8b_prefill", "paged_decode_b64"),
     "long": ("long_prefill_16k", "long_decode_131k"),
     "varlen": ("varlen_prefill_16seq", "paged_decode_b64"),
+    "chunked": ("chunked_prefill_paged", "paged_decode_b64"),
 }
 
 
 class PrefillCase:
-    """The prefill half of a step: dense (attn_fwd) or packed (attn_fwd_varlen)."""
+    """The prefill half of a step: dense (attn_fwd) or packed (attn_fwd_varlen); `--workload chunked` by a 512-token chunk of each of 8
+sequences against their paged cache of 1k-8k tokens (paged_attn_prefill)."""
 
     def __init__(self, name, seed, dev, fa, inputs, workloads):
         import torch
         self.name = name
         self.varlen = name in inputs.VARLEN_WORKLOADS
-        if self.varlen:
+        self.chunked = name in inputs.CHUNKED_WORKLOADS
+        if self.chunked:
+            sp = self.spec = inputs.CHUNKED_WORKLOADS[name]
+            ci = inputs.make_chunked(sp, seed=seed)
+            c = ci.cache
+            self.host_in = [ci.q, c.k_cache, c.v_cache, c.block_table, c.seq_lens, ci.cu_q]
+            lens_q = (ci.cu_q[1:] - ci.cu_q[:-1]).tolist()
+            ctx = c.seq_lens.tolist()
+            self.flops = sum(workloads.prefill_flops(1, sp.Hq, t, s_, sp.d, sp.causal) for t, s_ in zip(lens_q, ctx))
+            self.max_q, self.total_q, self.max_blocks = ci.max_q, int(ci.cu_q[-1]), c.block_table.shape[1]
+            self.dev_in = [t.to(dev) for t in self.host_in]
+            self.o = torch.empty_like(self.dev_in[0])
+            self.lse = torch.empty(sp.Hq, self.total_q, device=dev, dtype=torch.float32)
+            self.config = {**vars_of(sp), "context_lengths": ctx, "query_counts": lens_q}
+        elif self.varlen:
             sp = self.spec = inputs.VARLEN_WORKLOADS[name]
             vin = inputs.make_varlen(sp, seed=seed)
             self.host_in = [vin.q, vin.k, vin.v, vin.cu_q, vin.cu_k]
@@ -77,7 +94,11 @@ class PrefillCase:
 
     def call(self, stream):
         sp, fa = self.spec, self.fa
-        if self.varlen:
+        if self.chunked:
+            q, kc, vc, bt, sl, cq = self.dev_in
+            fa.paged_attn_prefill(q, kc, vc, bt, sl, cq, sp.B, sp.Hq, sp.Hkv, sp.d, sp.block_size, self.max_blocks,
+                                  self.max_q, self.total_q, sp.causal, sp.scale, self.o, self.lse, stream)
+        elif self.varlen:
             q, k, v, cq, ck = self.dev_in
             fa.attn_fwd_varlen(q, k, v, self.o, self.lse, cq, ck, sp.B, self.max_q, self.total_q, self.total_k,
                                sp.Hq, sp.Hkv, sp.d, sp.causal, sp.scale, stream)
@@ -205,6 +226,23 @@ def _cpu_prefill_varlen(pname, seed_offset, orc, inputs, workloads, f):
     return tp * sum(pairs) / max(sum(pairs[:n]), 1), flops, f"sequences {n}/{sp.B} (all {sp.Hq} heads)"
 
 
+def _cpu_prefill_chunked(pname, seed_offset, orc, inputs, workloads, f):
+    """Oracle time of a chunked paged prefill, from its first sequence,
+    scaled by visible pairs to all sequences."""
+    sp = inputs.CHUNKED_WORKLOADS[pname]
+    ci = inputs.make_chunked(sp, seed=sp.seed + seed_offset)
+    c = ci.cache
+    lq = (ci.cu_q[1:] - ci.cu_q[:-1]).tolist()
+    ctx = c.seq_lens.tolist()
+    t0 = time.perf_counter()
+    orc.paged_prefill(f(ci.q[:lq[0]]), f(c.k_cache), f(c.v_cache), c.block_table.numpy()[:1], ctx[:1],
+                      ci.cu_q.numpy()[:2], c.block_size, sp.scale, sp.causal)
+    tp = time.perf_counter() - t0
+    pairs = [workloads.visible_pairs(t, s_, sp.causal) for t, s_ in zip(lq, ctx)]
+    flops = sum(workloads.prefill_flops(1, sp.Hq, t, s_, sp.d, sp.causal) for t, s_ in zip(lq, ctx))
+    return tp * sum(pairs) / max(pairs[0], 1), flops, f"sequences 1/{sp.B} (all {sp.Hq} heads)"
+
+
 def cpu_baseline(pname, dname, peaks, seed_offset=0, budget_s=20.0):
     import torch
 
@@ -219,6 +257,8 @@ def cpu_baseline(pname, dname, peaks, seed_offset=0, budget_s=20.0):
     f = lambda t: t.to(torch.float64).numpy()  # noqa: E731
     if pname in inputs.VARLEN_WORKLOADS:
         t_prefill, flops, pdesc = _cpu_prefill_varlen(pname, seed_offset, orc, inputs, workloads, f)
+    elif pname in inputs.CHUNKED_WORKLOADS:
+        t_prefill, flops, pdesc = _cpu_prefill_chunked(pname, seed_offset, orc, inputs, workloads, f)
     else:
         t_prefill, flops, pdesc = _cpu_prefill_dense(pname, seed_offset, orc, inputs, workloads, f)
     ds = inputs.WORKLOADS[dname]
@@ -279,7 +319,8 @@ def main():
 
     ds = inputs.WORKLOADS[dname]
     # weak scaling: every rank runs its own batch (different seeds), no exchange
-    pspec = inputs.VARLEN_WORKLOADS.get(pname) or inputs.WORKLOADS[pname]
+    pspec = (inputs.VARLEN_WORKLOADS.get(pname) or inputs.CHUNKED_WORKLOADS.get(pname)
+             or inputs.WORKLOADS[pname])
     pre = PrefillCase(pname, dist_util.rank_seed(pspec.seed, rank), dev, fa, inputs, workloads)
     dinp = inputs.make_paged(ds, seed=dist_util.rank_seed(ds.seed, rank))
     qd_, kc, vc = dinp.q.to(dev), dinp.k_cache.to(dev), dinp.v_cache.to(dev)
@@ -438,7 +479,8 @@ def run_reference(args, pname, dname, peaks, peak_src, world):
         "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": est * 1e3, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic (same seeds as ours)",
-        "config": {"workload": f"{pname} + {dname}", "prefill": vars_of(inputs.VARLEN_WORKLOADS.get(pname) or inputs.WORKLOADS[pname]),
+        "config": {"workload": f"{pname} + {dname}", "prefill": vars_of(inputs.VARLEN_WORKLOADS.get(pname) or inputs.CHUNKED_WORKLOADS.get(pname)
+                                     or inputs.WORKLOADS[pname]),
                    "decode": vars_of(inputs.WORKLOADS[dname])},
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": info["cores"], "kind": "oracle",
                          "sample": info["sample"]},

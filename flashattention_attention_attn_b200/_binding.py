@@ -40,6 +40,9 @@ def library() -> ctypes.CDLL:
         lib.attn_fwd_varlen.argtypes = [vp, vp, vp, vp, vp, vp, vp, c_int, c_int, c_int, c_int, c_int, c_int, c_int,
                                         c_int, c_float, vp]
         lib.attn_fwd_varlen.restype = c_int
+        lib.paged_attn_prefill.argtypes = [vp, vp, vp, vp, vp, vp, c_int, c_int, c_int, c_int, c_int, c_int, c_int,
+                                           c_int, c_int, c_float, vp, vp, vp]
+        lib.paged_attn_prefill.restype = c_int
         lib.paged_attn_decode.argtypes = [vp, vp, vp, vp, vp, c_int, c_int, c_int, c_int, c_int, c_int, c_int,
                                           vp, vp]
         lib.paged_attn_decode.restype = c_int
@@ -97,6 +100,17 @@ def attn_fwd_varlen(q, k, v, o, lse, cu_seqlens_q, cu_seqlens_k, B, max_seqlen_q
                                    int(Hq), int(Hkv), int(d), int(bool(causal)), float(scale), _stream(stream))
     if rc != ATTN_OK:
         raise AttnError(rc, "attn_fwd_varlen")
+
+
+def paged_attn_prefill(q, k_cache, v_cache, block_table, seq_lens, cu_seqlens_q, B, Hq, Hkv, d, block_size,
+                       max_blocks, max_seqlen_q, total_q, causal, scale, o, lse, stream=None) -> None:
+    """Chunked prefill against the paged cache (see attn.h)."""
+    rc = library().paged_attn_prefill(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_table), _ptr(seq_lens),
+                                      _ptr(cu_seqlens_q), int(B), int(Hq), int(Hkv), int(d), int(block_size),
+                                      int(max_blocks), int(max_seqlen_q), int(total_q), int(bool(causal)),
+                                      float(scale), _ptr(o), _ptr(lse), _stream(stream))
+    if rc != ATTN_OK:
+        raise AttnError(rc, "paged_attn_prefill")
 
 
 def paged_attn_decode(q, k_cache, v_cache, block_table, seq_lens, B, Hq, Hkv, d, block_size, max_blocks,

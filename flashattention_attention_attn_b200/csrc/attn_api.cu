@@ -69,7 +69,7 @@ int probe_device(int dev, DeviceState** out) {
       st.status = ATTN_ERR_UNSUPPORTED;
     } else {
       cudaFuncAttributes fa;
-      if (cudaFuncGetAttributes(&fa, prefill::prefill_fwd_sm100<128, false>) != cudaSuccess) {
+      if (cudaFuncGetAttributes(&fa, prefill::prefill_fwd_sm100<128, prefill::kDense>) != cudaSuccess) {
         cudaGetLastError();
         st.status = ATTN_ERR_UNSUPPORTED;  // no sm_100a image for this device
       } else if (encode_tiled() == nullptr) {
@@ -93,10 +93,12 @@ int prepare_device(int dev, DeviceState* st) {
     const void* fn;
     size_t bytes;
   } kernels[] = {
-      {reinterpret_cast<const void*>(prefill::prefill_fwd_sm100<64, false>), prefill::smem_bytes<64>()},
-      {reinterpret_cast<const void*>(prefill::prefill_fwd_sm100<128, false>), prefill::smem_bytes<128>()},
-      {reinterpret_cast<const void*>(prefill::prefill_fwd_sm100<64, true>), prefill::smem_bytes<64>()},
-      {reinterpret_cast<const void*>(prefill::prefill_fwd_sm100<128, true>), prefill::smem_bytes<128>()},
+      {reinterpret_cast<const void*>(prefill::prefill_fwd_sm100<64, prefill::kDense>), prefill::smem_bytes<64>()},
+      {reinterpret_cast<const void*>(prefill::prefill_fwd_sm100<128, prefill::kDense>), prefill::smem_bytes<128>()},
+      {reinterpret_cast<const void*>(prefill::prefill_fwd_sm100<64, prefill::kVarlen>), prefill::smem_bytes<64>()},
+      {reinterpret_cast<const void*>(prefill::prefill_fwd_sm100<128, prefill::kVarlen>), prefill::smem_bytes<128>()},
+      {reinterpret_cast<const void*>(prefill::prefill_fwd_sm100<64, prefill::kPaged>), prefill::smem_bytes<64>()},
+      {reinterpret_cast<const void*>(prefill::prefill_fwd_sm100<128, prefill::kPaged>), prefill::smem_bytes<128>()},
       {reinterpret_cast<const void*>(decode::paged_decode_split<64>), decode::smem_bytes<64>()},
       {reinterpret_cast<const void*>(decode::paged_decode_split<128>), decode::smem_bytes<128>()},
   };
@@ -188,7 +190,7 @@ int launch_prefill(const void* q, const void* k, const void* v, void* o, float* 
   p.num_mblocks = (T + 2 * prefill::kBM - 1) / (2 * prefill::kBM);
   const long long grid = static_cast<long long>(p.num_mblocks) * Hq * B;
   if (grid > 0x7fffffffLL) return ATTN_ERR_UNSUPPORTED;
-  prefill::prefill_fwd_sm100<D, false><<<static_cast<unsigned>(grid), prefill::kThreads,
+  prefill::prefill_fwd_sm100<D, prefill::kDense><<<static_cast<unsigned>(grid), prefill::kThreads,
                                          prefill::smem_bytes<D>(), stream>>>(mq, mk, mv, mo, p);
   return launch_status();
 }
@@ -221,8 +223,41 @@ int launch_prefill_varlen(const void* q, const void* k, const void* v, void* o, 
   p.num_mblocks = (max_q + 2 * prefill::kBM - 1) / (2 * prefill::kBM);
   const long long grid = static_cast<long long>(p.num_mblocks) * Hq * B;
   if (grid > 0x7fffffffLL) return ATTN_ERR_UNSUPPORTED;
-  prefill::prefill_fwd_sm100<D, true><<<static_cast<unsigned>(grid), prefill::kThreads,
+  prefill::prefill_fwd_sm100<D, prefill::kVarlen><<<static_cast<unsigned>(grid), prefill::kThreads,
                                         prefill::smem_bytes<D>(), stream>>>(mq, mk, mv, mo, p);
+  return launch_status();
+}
+
+// Chunked prefill against the paged cache: packed queries as in varlen,
+// keys and values gathered through the block table from the pool maps.
+template <int D>
+int launch_prefill_paged(const void* q, const void* kc, const void* vc, const int32_t* table, const int32_t* lens,
+                         const int32_t* cu_q, void* o, float* lse, int B, int max_q, int total_q, int Hq, int Hkv,
+                         int max_blocks, int causal, float scale, cudaStream_t stream) {
+  CUtensorMap mq, mk, mv, mo;
+  if (make_map_bthd(&mq, q, 1, total_q, Hq, D) || make_map_pool(&mk, kc, Hkv, D) || make_map_pool(&mv, vc, Hkv, D) ||
+      make_map_bthd(&mo, o, 1, total_q, Hq, D))
+    return ATTN_ERR_CUDA;
+  prefill::Params p;
+  std::memset(&p, 0, sizeof(p));
+  p.lse = lse;
+  p.o = static_cast<__nv_bfloat16*>(o);
+  p.cu_q = cu_q;
+  p.block_table = table;
+  p.seq_lens = lens;
+  p.max_blocks = max_blocks;
+  p.B = B;
+  p.Hq = Hq;
+  p.Hkv = Hkv;
+  p.T = max_q;
+  p.total_q = total_q;
+  p.causal = causal ? 1 : 0;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  p.num_mblocks = (max_q + 2 * prefill::kBM - 1) / (2 * prefill::kBM);
+  const long long grid = static_cast<long long>(p.num_mblocks) * Hq * B;
+  if (grid > 0x7fffffffLL) return ATTN_ERR_UNSUPPORTED;
+  prefill::prefill_fwd_sm100<D, prefill::kPaged><<<static_cast<unsigned>(grid), prefill::kThreads,
+                                                   prefill::smem_bytes<D>(), stream>>>(mq, mk, mv, mo, p);
   return launch_status();
 }
 
@@ -397,6 +432,37 @@ extern "C" int attn_fwd_varlen(const void* q, const void* k, const void* v, void
                                      Hq, Hkv, causal, scale, stream);
   return launch_prefill_varlen<128>(q, k, v, o, lse, cu_seqlens_q, cu_seqlens_k, B, max_seqlen_q, total_q, total_k,
                                     Hq, Hkv, causal, scale, stream);
+}
+
+extern "C" int paged_attn_prefill(const void* q, const void* k_cache, const void* v_cache,
+                                  const int32_t* block_table, const int32_t* seq_lens, const int32_t* cu_seqlens_q,
+                                  int B, int Hq, int Hkv, int d, int block_size, int max_blocks, int max_seqlen_q,
+                                  int total_q, int causal, float scale, void* o, float* lse, attn_stream_t stream_) {
+  cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+  if (B < 0 || Hq <= 0 || Hkv <= 0 || d <= 0 || block_size <= 0 || max_seqlen_q < 0 || total_q < 0)
+    return ATTN_ERR_INVALID_ARG;
+  if (Hq % Hkv != 0) return ATTN_ERR_INVALID_ARG;
+  if (!(scale > 0.f) || !std::isfinite(scale)) return ATTN_ERR_INVALID_ARG;
+  if (B == 0 || total_q == 0 || max_seqlen_q == 0) return ATTN_OK;
+  if (max_blocks <= 0) return ATTN_ERR_INVALID_ARG;
+  if (q == nullptr || k_cache == nullptr || v_cache == nullptr || block_table == nullptr || seq_lens == nullptr ||
+      cu_seqlens_q == nullptr || o == nullptr)
+    return ATTN_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return ATTN_ERR_UNSUPPORTED;
+  if (block_size != decode::kBlock) return ATTN_ERR_UNSUPPORTED;
+  if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(o)) return ATTN_ERR_UNSUPPORTED;
+  if ((lse != nullptr && (reinterpret_cast<uintptr_t>(lse) & 3u)) ||
+      (reinterpret_cast<uintptr_t>(block_table) & 3u) || (reinterpret_cast<uintptr_t>(seq_lens) & 3u) ||
+      (reinterpret_cast<uintptr_t>(cu_seqlens_q) & 3u))
+    return ATTN_ERR_UNSUPPORTED;
+  DeviceState* st = nullptr;
+  int rc = current_device_state(&st);
+  if (rc != ATTN_OK) return rc;
+  if (d == 64)
+    return launch_prefill_paged<64>(q, k_cache, v_cache, block_table, seq_lens, cu_seqlens_q, o, lse, B,
+                                    max_seqlen_q, total_q, Hq, Hkv, max_blocks, causal, scale, stream);
+  return launch_prefill_paged<128>(q, k_cache, v_cache, block_table, seq_lens, cu_seqlens_q, o, lse, B,
+                                   max_seqlen_q, total_q, Hq, Hkv, max_blocks, causal, scale, stream);
 }
 
 extern "C" int paged_attn_decode(const void* q, const void* k_cache, const void* v_cache,

@@ -113,6 +113,7 @@ struct __align__(1024) Smem {
   uint64_t v_full[C::kStages], v_empty[C::kStages];
   uint64_t s_full[2], p_full[2][kPChunks], o_full[2];
   uint64_t mma_done;
+  uint64_t v_tail;  // paged: V tile holding the sequence end, before its tail is cleared
   uint32_t tmem_base;
   int abort_flag;
 };
@@ -122,11 +123,19 @@ constexpr size_t smem_bytes() {
   return sizeof(Smem<D>) + 1024;  // + slack to align the dynamic base to 1024
 }
 
+// How queries and keys are laid out.
+constexpr int kDense = 0;   // [B, T, H, D] / [B, S, H, D]
+constexpr int kVarlen = 1;  // packed [total, H, D], offsets from cu_q / cu_k
+constexpr int kPaged = 2;   // packed queries; keys and values in a paged pool
+
 struct Params {
-  float* lse;             // [B, Hq, T] (dense) / [Hq, total_q] (varlen), or nullptr
-  __nv_bfloat16* o;       // output base (row stores of ragged varlen tiles)
-  const int32_t* cu_q;    // varlen: [B + 1] prefix sums of query lengths
+  float* lse;             // [B, Hq, T] (dense) / [Hq, total_q] (packed), or nullptr
+  __nv_bfloat16* o;       // output base (row stores of ragged packed tiles)
+  const int32_t* cu_q;    // packed: [B + 1] prefix sums of query lengths
   const int32_t* cu_k;    // varlen: [B + 1] prefix sums of key lengths
+  const int32_t* block_table;  // paged: [B, max_blocks] physical 16-token blocks
+  const int32_t* seq_lens;     // paged: [B] cached tokens (keys) per sequence
+  int max_blocks;
   int B, Hq, Hkv, T, S;   // dense: T, S; varlen: T = max query length
   int total_q;            // varlen: rows of the packed query tensor
   int causal;
@@ -145,10 +154,12 @@ __device__ __forceinline__ int kv_tiles_for(int r0, int T, int S, int causal) {
   return kmax / kBN + 1;
 }
 
-// VARLEN: packed sequences (no padding).  The tensor maps then cover
-// [total, H, D] as batch 1, and each CTA takes its sequence's row offsets
-// and lengths from cu_q / cu_k.
-template <int D, bool VARLEN>
+// MODE kVarlen / kPaged: packed sequences (no padding).  The query / output
+// maps then cover [total, H, D] as batch 1 and each CTA takes its sequence's
+// row offset and length from cu_q.  kVarlen takes key rows from cu_k the
+// same way; kPaged reads every 128-key tile as eight 16-token blocks through
+// the block table (pool maps of [tokens, Hkv * D], box 64 x 16).
+template <int D, int MODE>
 __global__ void __launch_bounds__(kThreads, 1)
     prefill_fwd_sm100(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                       const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
@@ -169,12 +180,17 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int b = rem / p.Hq;
   const int hk = h / (p.Hq / p.Hkv);
   const int m0 = mb * 2 * kBM;
+  constexpr bool VARLEN = MODE != kDense;  // packed queries and outputs
   int T = p.T, S = p.S, qoff = 0, koff = 0, bc = b;  // bc: batch coordinate of the maps
   if constexpr (VARLEN) {
     qoff = p.cu_q[b];
     T = p.cu_q[b + 1] - qoff;
-    koff = p.cu_k[b];
-    S = p.cu_k[b + 1] - koff;
+    if constexpr (MODE == kPaged) {
+      S = p.seq_lens[b];
+    } else {
+      koff = p.cu_k[b];
+      S = p.cu_k[b + 1] - koff;
+    }
     bc = 0;
     if (m0 >= T) return;  // this query block lies past the sequence (uniform over the CTA)
   }
@@ -196,6 +212,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&sm.v_empty[s], 1);
     }
     mbar_init(&sm.mma_done, 1);
+    mbar_init(&sm.v_tail, 1);
     sm.abort_flag = 0;
     fence_mbarrier_init();
   }
@@ -211,41 +228,105 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (warp == kWarpLoad) {
     // ------------------------------ producer ------------------------------
+    // The whole warp runs the loop (paged mode loads block ids in parallel);
+    // lane 0 waits on the barriers and issues the copies.
     if (lane == 0) {
       tma_prefetch_desc(&tmQ);
       tma_prefetch_desc(&tmK);
       tma_prefetch_desc(&tmV);
-      const int nt[2] = {n0, n1};
+    }
+    const int nt[2] = {n0, n1};
+    if (lane == 0) {
       for (int t = 0; t < 2; ++t) {
         if (nt[t] == 0) continue;
         mbar_arrive_expect_tx(&sm.q_full[t], C::kTileBytes);
         for (int c = 0; c < C::kChunks; ++c)
           tma_load_4d(sm.q[t][c], &tmQ, &sm.q_full[t], c * 64, h, qoff + m0 + t * kBM, bc);
       }
-      int k_issued = 0, v_issued = 0;  // K / V tiles whose loads were issued
-      for (int j = 0; j < n_max; ++j) {
-        const int s = j % C::kStages;
-        const uint32_t ph = (j / C::kStages) & 1;
-        if (!mbar_wait(&sm.k_empty[s], ph ^ 1, abort_flag)) break;
-        mbar_arrive_expect_tx(&sm.k_full[s], C::kTileBytes);
-        for (int c = 0; c < C::kChunks; ++c)
-          tma_load_4d(sm.k[s][c], &tmK, &sm.k_full[s], c * 64, hk, koff + j * kBN, bc);
-        k_issued = j + 1;
-        if (!mbar_wait(&sm.v_empty[s], ph ^ 1, abort_flag)) break;
-        mbar_arrive_expect_tx(&sm.v_full[s], C::kTileBytes);
-        for (int c = 0; c < C::kChunks; ++c)
-          tma_load_4d(sm.v[s][c], &tmV, &sm.v_full[s], c * 64, hk, koff + j * kBN, bc);
-        v_issued = j + 1;
+    }
+    int k_issued = 0, v_issued = 0;  // K / V tiles whose loads were issued
+    bool tail_issued = false;
+    for (int j = 0; j < n_max; ++j) {
+      const int s = j % C::kStages;
+      const uint32_t ph = (j / C::kStages) & 1;
+      int nblk = kBN / 16;   // 16-token blocks loaded into this tile
+      int valid = kBN;       // keys of this tile inside the sequence
+      int ids[kBN / 16];
+      if constexpr (MODE == kPaged) {
+        valid = min(kBN, S - j * kBN);
+        nblk = (valid + 15) / 16;
+        const int mine = (lane < nblk) ? __ldg(p.block_table + static_cast<size_t>(b) * p.max_blocks +
+                                               j * (kBN / 16) + lane)
+                                       : 0;
+#pragma unroll
+        for (int i = 0; i < kBN / 16; ++i) ids[i] = __shfl_sync(0xffffffffu, mine, i);
       }
-      if (*abort_flag) {
-        // Let the copies already issued land before shared memory is released.
-        for (int t = 0; t < 2; ++t)
-          if (nt[t] > 0) mbar_wait_drain(&sm.q_full[t], 0);
-        for (int j = max(0, k_issued - C::kStages); j < k_issued; ++j)
-          mbar_wait_drain(&sm.k_full[j % C::kStages], (j / C::kStages) & 1);
-        for (int j = max(0, v_issued - C::kStages); j < v_issued; ++j)
-          mbar_wait_drain(&sm.v_full[j % C::kStages], (j / C::kStages) & 1);
+      const uint32_t tile_bytes = static_cast<uint32_t>(nblk) * 16 * D * 2;
+      bool ok = true;
+      if (lane == 0) {
+        ok = mbar_wait(&sm.k_empty[s], ph ^ 1, abort_flag);
+        if (ok) {
+          mbar_arrive_expect_tx(&sm.k_full[s], tile_bytes);
+          for (int c = 0; c < C::kChunks; ++c) {
+            if constexpr (MODE == kPaged) {
+              for (int i = 0; i < nblk; ++i)
+                tma_load_2d(reinterpret_cast<uint8_t*>(sm.k[s][c]) + i * 16 * 128, &tmK, &sm.k_full[s],
+                            hk * D + c * 64, ids[i] * 16);
+            } else {
+              tma_load_4d(sm.k[s][c], &tmK, &sm.k_full[s], c * 64, hk, koff + j * kBN, bc);
+            }
+          }
+          k_issued = j + 1;
+          ok = mbar_wait(&sm.v_empty[s], ph ^ 1, abort_flag);
+        }
       }
+      if (!__shfl_sync(0xffffffffu, ok ? 1 : 0, 0)) break;
+      if (MODE == kPaged && valid < kBN) {
+        // The tile holding the sequence end: its V copy completes on v_tail;
+        // then the rows past the end (pool slots that may hold anything,
+        // even NaN, and blocks not loaded) are cleared so that a zero weight
+        // cannot meet a NaN, and only then is the tile handed to the MMA.
+        if (lane == 0) {
+          mbar_arrive_expect_tx(&sm.v_tail, tile_bytes);
+          for (int c = 0; c < C::kChunks; ++c)
+            for (int i = 0; i < nblk; ++i)
+              tma_load_2d(reinterpret_cast<uint8_t*>(sm.v[s][c]) + i * 16 * 128, &tmV, &sm.v_tail,
+                          hk * D + c * 64, ids[i] * 16);
+          tail_issued = true;
+        }
+        ok = __shfl_sync(0xffffffffu, mbar_wait(&sm.v_tail, 0, abort_flag) ? 1 : 0, 0) != 0;
+        if (!ok) break;
+        for (int i = lane; i < (kBN - valid) * C::kChunks * 8; i += 32) {
+          const int unit = i & 7, c = (i >> 3) % C::kChunks, r = valid + (i >> 3) / C::kChunks;
+          *reinterpret_cast<uint4*>(reinterpret_cast<uint8_t*>(sm.v[s][c]) + r * 128 + unit * 16) =
+              make_uint4(0u, 0u, 0u, 0u);
+        }
+        fence_proxy_async_smem();  // the generic writes before the tensor core reads the tile
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&sm.v_full[s]);
+      } else if (lane == 0) {
+        mbar_arrive_expect_tx(&sm.v_full[s], tile_bytes);
+        for (int c = 0; c < C::kChunks; ++c) {
+          if constexpr (MODE == kPaged) {
+            for (int i = 0; i < nblk; ++i)
+              tma_load_2d(reinterpret_cast<uint8_t*>(sm.v[s][c]) + i * 16 * 128, &tmV, &sm.v_full[s],
+                          hk * D + c * 64, ids[i] * 16);
+          } else {
+            tma_load_4d(sm.v[s][c], &tmV, &sm.v_full[s], c * 64, hk, koff + j * kBN, bc);
+          }
+        }
+      }
+      v_issued = j + 1;
+    }
+    if (lane == 0 && *abort_flag) {
+      // Let the copies already issued land before shared memory is released.
+      for (int t = 0; t < 2; ++t)
+        if (nt[t] > 0) mbar_wait_drain(&sm.q_full[t], 0);
+      for (int j = max(0, k_issued - C::kStages); j < k_issued; ++j)
+        mbar_wait_drain(&sm.k_full[j % C::kStages], (j / C::kStages) & 1);
+      for (int j = max(0, v_issued - C::kStages); j < v_issued; ++j)
+        mbar_wait_drain(&sm.v_full[j % C::kStages], (j / C::kStages) & 1);
+      if (tail_issued) mbar_wait_drain(&sm.v_tail, 0);
     }
   } else if (warp == kWarpMma) {
     // ---------------------------- MMA issuer ------------------------------

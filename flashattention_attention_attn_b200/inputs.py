@@ -222,3 +222,66 @@ def make_varlen(spec: VarlenSpec, q_lens=None, k_lens=None, seed: int | None = N
     k = _randn_bf16(gen, (int(cu_k[-1]), s.Hkv, s.d))
     v = _randn_bf16(gen, (int(cu_k[-1]), s.Hkv, s.d))
     return VarlenInputs(q=q, k=k, v=v, cu_q=cu_q, cu_k=cu_k)
+
+
+@dataclass(frozen=True)
+class ChunkedSpec:
+    """Chunked prefill against a paged cache: each sequence has ctx tokens in
+    the cache, the last q_len of which are the new queries."""
+    B: int
+    Hq: int
+    Hkv: int
+    d: int
+    block_size: int
+    max_blocks: int
+    ctx_lo: int
+    ctx_hi: int
+    q_lo: int
+    q_hi: int
+    causal: bool = True
+    seed: int = 0
+
+    @property
+    def scale(self) -> float:
+        return 1.0 / (self.d ** 0.5)
+
+
+# 8 Llama3-8B-shaped sequences with 1k..8k cached tokens, a new chunk of 512
+CHUNKED_WORKLOADS = {
+    "chunked_prefill_paged": ChunkedSpec(B=8, Hq=32, Hkv=8, d=128, block_size=16, max_blocks=512, ctx_lo=1024,
+                                         ctx_hi=8192, q_lo=512, q_hi=512, causal=True, seed=1006),
+}
+
+
+@dataclass
+class ChunkedInputs:
+    q: torch.Tensor        # [total_q, Hq, d] bf16
+    cu_q: torch.Tensor     # [B + 1] int32
+    cache: PagedInputs     # pool, block table, seq_lens (its q is unused)
+
+    @property
+    def max_q(self) -> int:
+        return int((self.cu_q[1:] - self.cu_q[:-1]).max()) if self.cu_q.numel() > 1 else 0
+
+
+def make_chunked(spec: ChunkedSpec, ctx_lens=None, q_lens=None, seed: int | None = None) -> ChunkedInputs:
+    """Draw order: context lengths (uniform in [ctx_lo, ctx_hi] unless given),
+    query counts (uniform in [q_lo, q_hi], at most the context, unless
+    given), then the paged cache as make_paged draws it (physical-id
+    permutation, a decode q that is not used, the K pool, the V pool), then
+    the queries."""
+    s = spec
+    gen = torch.Generator(device="cpu").manual_seed(s.seed if seed is None else seed)
+    if ctx_lens is None:
+        ctx_lens = torch.randint(s.ctx_lo, s.ctx_hi + 1, (s.B,), generator=gen, dtype=torch.int64).tolist()
+    if q_lens is None:
+        q_lens = torch.randint(s.q_lo, s.q_hi + 1, (s.B,), generator=gen, dtype=torch.int64).tolist()
+    ctx_lens = [int(x) for x in ctx_lens]
+    q_lens = [min(int(t), c) for t, c in zip(q_lens, ctx_lens)]
+    dspec = DecodeSpec(B=s.B, Hq=s.Hq, Hkv=s.Hkv, d=s.d, block_size=s.block_size, max_blocks=s.max_blocks,
+                       ctx_lo=0, ctx_hi=0, seed=int(torch.randint(0, 2 ** 31 - 1, (1,), generator=gen)))
+    cache = make_paged(dspec, seq_lens=ctx_lens)
+    cu_q = torch.zeros(s.B + 1, dtype=torch.int32)
+    cu_q[1:] = torch.cumsum(torch.tensor(q_lens, dtype=torch.int64), 0).to(torch.int32)
+    q = _randn_bf16(gen, (int(cu_q[-1]), s.Hq, s.d))
+    return ChunkedInputs(q=q, cu_q=cu_q, cache=cache)

@@ -180,6 +180,36 @@ int attn_read_device_status(int* out, int clear);
 int attn_selftest_bounded_wait(attn_stream_t stream);
 
 /*
+ * paged_attn_prefill - chunked prefill against the paged KV cache: several
+ * new query tokens per sequence attend to that sequence's paged context
+ * (the paged cache and its block-table translation of the page "Snelle
+ * attention-kernels en operatorfusie versnellen AI-modellen", section
+ * "FlashAttention-type aandacht en gepagineerde aandacht", combined with the
+ * blockwise prefill of attn_fwd).
+ *
+ *   q            [total_q, Hq, d] bf16: the new tokens of the B sequences,
+ *                back to back (rows cu_seqlens_q[b] .. cu_seqlens_q[b+1])
+ *   k_cache, v_cache, block_table: as paged_attn_decode
+ *   seq_lens     [B] int32: tokens in the cache for sequence b, the new
+ *                tokens included (they are the last T_b of them)
+ *   cu_seqlens_q [B + 1] int32 prefix sums of the query counts T_b
+ *   o            [total_q, Hq, d] bf16 (written); lse [Hq, total_q] fp32 or NULL
+ *
+ *   Query row i of sequence b sits at position seq_lens[b] - T_b + i; with
+ *   causal != 0 it sees the keys at positions <= its own (bottom-right
+ *   alignment of attn_fwd with T = T_b, S = seq_lens[b]); otherwise all
+ *   seq_lens[b] keys.  Pool slots past the sequence end may hold anything.
+ *   max_seqlen_q must be >= every T_b.
+ *   Supported: d in {64, 128}; block_size == 16; Hq % Hkv == 0; sm_100.
+ *   Errors: as paged_attn_decode.
+ */
+int paged_attn_prefill(const void* q, const void* k_cache, const void* v_cache,
+                       const int32_t* block_table, const int32_t* seq_lens, const int32_t* cu_seqlens_q,
+                       int B, int Hq, int Hkv, int d, int block_size, int max_blocks,
+                       int max_seqlen_q, int total_q, int causal, float scale,
+                       void* o, float* lse, attn_stream_t stream);
+
+/*
  * paged_attn_decode_noalloc - paged_attn_decode for callers that must not
  * allocate device memory during the call.
  *

@@ -4,6 +4,7 @@ from .fp64_attention import (  # noqa: F401
     attention_varlen,
     gather_paged_kv,
     paged_decode,
+    paged_prefill,
     softmax_rows,
     split_paged_decode,
     visible_key_count,

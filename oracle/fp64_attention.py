@@ -52,6 +52,7 @@ __all__ = [
     "attention_varlen",
     "gather_paged_kv",
     "paged_decode",
+    "paged_prefill",
     "split_paged_decode",
 ]
 
@@ -192,6 +193,33 @@ def paged_decode(q, k_cache, v_cache, block_table, seq_lens, block_size: int, sc
         ob, lb = attention(q[b][None, None], Kb[None], Vb[None], scale, causal=False)
         O[b] = ob[0, 0]
         LSE[b] = lb[0, :, 0]
+    return O, LSE
+
+
+def paged_prefill(q, k_cache, v_cache, block_table, seq_lens, cu_q, block_size: int, scale: float, causal: bool):
+    """Chunked prefill against a paged cache, fp64.
+
+    q: [total_q, Hq, d] (the new tokens of every sequence, back to back,
+    rows cu_q[b]..cu_q[b+1]); the cache holds seq_lens[b] tokens of
+    sequence b, the new ones included as its last T_b tokens.  The logical
+    K/V are gathered through the block table, then `attention` is applied
+    with T = T_b and S = seq_lens[b] (bottom-right causal alignment: the new
+    token i sits at position S - T + i).  Returns O [total_q, Hq, d] and
+    LSE [Hq, total_q].
+    """
+    q = np.asarray(q, dtype=np.float64)
+    total_q, Hq, d = q.shape
+    O = np.zeros((total_q, Hq, d))
+    LSE = np.full((Hq, total_q), -np.inf)
+    for b in range(len(cu_q) - 1):
+        q0, q1 = int(cu_q[b]), int(cu_q[b + 1])
+        L = int(seq_lens[b])
+        if q1 == q0:
+            continue
+        Kb, Vb = gather_paged_kv(k_cache, v_cache, block_table[b], L, block_size)
+        ob, lb = attention(q[None, q0:q1], Kb[None], Vb[None], scale, causal)
+        O[q0:q1] = ob[0]
+        LSE[:, q0:q1] = lb[0]
     return O, LSE
 
 

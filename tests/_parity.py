@@ -91,3 +91,26 @@ def run_varlen(inp, causal, scale, max_q=None):
 
 def oracle_varlen(inp, causal, scale):
     return orc.attention_varlen(f64(inp.q), f64(inp.k), f64(inp.v), inp.cu_q.numpy(), inp.cu_k.numpy(), scale, causal)
+
+
+def run_chunked(inp, causal, scale):
+    import flashattention_attention_attn_b200 as fa
+    total_q, Hq, d = inp.q.shape
+    c = inp.cache
+    Hkv = c.k_cache.shape[2]
+    B = inp.cu_q.numel() - 1
+    dq = inp.q.cuda()
+    o = torch.full_like(dq, float("nan"))
+    lse = torch.full((Hq, total_q), float("nan"), device="cuda", dtype=torch.float32)
+    fa.paged_attn_prefill(dq, c.k_cache.cuda(), c.v_cache.cuda(), c.block_table.cuda(), c.seq_lens.cuda(),
+                          inp.cu_q.cuda(), B, Hq, Hkv, d, c.block_size, c.block_table.shape[1], inp.max_q, total_q,
+                          causal, scale, o, lse)
+    torch.cuda.synchronize()
+    assert fa.attn_read_device_status(clear=True) == 0
+    return o.cpu(), lse.cpu()
+
+
+def oracle_chunked(inp, causal, scale):
+    c = inp.cache
+    return orc.paged_prefill(f64(inp.q), f64(c.k_cache), f64(c.v_cache), c.block_table.numpy(), c.seq_lens.numpy(),
+                             inp.cu_q.numpy(), c.block_size, scale, causal)

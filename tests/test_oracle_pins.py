@@ -312,3 +312,44 @@ def test_varlen_sequences_do_not_see_each_other():
     O2, L2 = orc.attention_varlen(q, k2, v2, cu_q, cu_k, 0.3, True)
     np.testing.assert_array_equal(O1[:cu_q[1]], O2[:cu_q[1]])
     np.testing.assert_array_equal(L1[:, :cu_q[1]], L2[:, :cu_q[1]])
+
+
+def _chunked_case(seed, ctx, qlens, bs=4, max_blocks=10, Hq=4, Hkv=2, d=8):
+    rng = np.random.default_rng(seed)
+    nblk = [(c + bs - 1) // bs for c in ctx]
+    pool = sum(nblk) + 2
+    perm = rng.permutation(pool)
+    table = -np.ones((len(ctx), max_blocks), dtype=np.int32)
+    at = 0
+    for b, n in enumerate(nblk):
+        table[b, :n] = perm[at:at + n]
+        at += n
+    cu_q = np.concatenate([[0], np.cumsum(qlens)]).astype(np.int64)
+    q = rng.standard_normal((cu_q[-1], Hq, d))
+    kc = rng.standard_normal((pool, bs, Hkv, d))
+    vc = rng.standard_normal((pool, bs, Hkv, d))
+    return q, kc, vc, table, np.array(ctx), cu_q, bs
+
+
+def test_paged_prefill_one_token_is_decode():
+    q, kc, vc, table, lens, cu_q, bs = _chunked_case(50, [7, 13, 1, 30], [1, 1, 1, 1])
+    O, L = orc.paged_prefill(q, kc, vc, table, lens, cu_q, bs, 0.3, True)
+    Od, Ld = orc.paged_decode(q, kc, vc, table, lens, bs, 0.3)
+    np.testing.assert_allclose(O, Od, rtol=0, atol=1e-12)
+    np.testing.assert_allclose(L, Ld.T, rtol=0, atol=1e-12)
+
+
+def test_paged_prefill_equals_contiguous_tail_rows():
+    """The new tokens are the last rows of a causal prefill over the whole
+    context written out position by position (independent of the gather)."""
+    ctx, qlens = [9, 17, 30], [4, 17, 3]
+    q, kc, vc, table, lens, cu_q, bs = _chunked_case(51, ctx, qlens)
+    O, L = orc.paged_prefill(q, kc, vc, table, lens, cu_q, bs, 0.3, True)
+    for b, (c, t) in enumerate(zip(ctx, qlens)):
+        K = np.stack([kc[table[b, p // bs], p % bs] for p in range(c)])[None]
+        V = np.stack([vc[table[b, p // bs], p % bs] for p in range(c)])[None]
+        Q = np.zeros((1, c, q.shape[1], q.shape[2]))
+        Q[0, c - t:] = q[cu_q[b]:cu_q[b + 1]]
+        Of, Lf = orc.attention(Q, K, V, 0.3, True)
+        np.testing.assert_allclose(O[cu_q[b]:cu_q[b + 1]], Of[0, c - t:], rtol=0, atol=1e-12)
+        np.testing.assert_allclose(L[:, cu_q[b]:cu_q[b + 1]], Lf[0, :, c - t:], rtol=0, atol=1e-12)
