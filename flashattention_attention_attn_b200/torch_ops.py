@@ -1,0 +1,54 @@
+"""torch custom ops over the C ABI, so that the kernels compose with
+torch.compile (no graph break: the ops have fake/meta implementations that
+give output shapes without running anything) and with CUDA-graph capture.
+
+    import flashattention_attention_attn_b200.torch_ops  # registers the ops
+    o, lse = torch.ops.fa_b200.attn_fwd(q, k, v, causal, scale)
+    o = torch.ops.fa_b200.paged_attn_decode(q, k_cache, v_cache, block_table, seq_lens, num_splits)
+
+The op bodies only allocate the outputs and call the library on the current
+stream; there is no other path.  Shapes follow include/attn.h:
+q [B,T,Hq,d], k/v [B,S,Hkv,d] -> o [B,T,Hq,d], lse [B,Hq,T];
+decode q [B,Hq,d], caches [num_blocks,16,Hkv,d], block_table [B,max_blocks],
+seq_lens [B] -> o [B,Hq,d].
+"""
+
+from __future__ import annotations
+
+import torch
+
+from . import _binding
+
+
+@torch.library.custom_op("fa_b200::attn_fwd", mutates_args=())
+def attn_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, causal: bool,
+             scale: float) -> tuple[torch.Tensor, torch.Tensor]:
+    B, T, Hq, d = q.shape
+    S, Hkv = k.shape[1], k.shape[2]
+    o = torch.empty_like(q)
+    lse = torch.empty((B, Hq, T), device=q.device, dtype=torch.float32)
+    _binding.attn_fwd(q, k, v, o, lse, B, Hq, Hkv, T, S, d, causal, scale,
+                      torch.cuda.current_stream(q.device))
+    return o, lse
+
+
+@attn_fwd.register_fake
+def _(q, k, v, causal, scale):
+    B, T, Hq, _ = q.shape
+    return torch.empty_like(q), q.new_empty((B, Hq, T), dtype=torch.float32)
+
+
+@torch.library.custom_op("fa_b200::paged_attn_decode", mutates_args=())
+def paged_attn_decode(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor, block_table: torch.Tensor,
+                      seq_lens: torch.Tensor, num_splits: int) -> torch.Tensor:
+    B, Hq, d = q.shape
+    Hkv, block_size = k_cache.shape[2], k_cache.shape[1]
+    o = torch.empty_like(q)
+    _binding.paged_attn_decode(q, k_cache, v_cache, block_table, seq_lens, B, Hq, Hkv, d, block_size,
+                               block_table.shape[1], num_splits, o, torch.cuda.current_stream(q.device))
+    return o
+
+
+@paged_attn_decode.register_fake
+def _(q, k_cache, v_cache, block_table, seq_lens, num_splits):
+    return torch.empty_like(q)

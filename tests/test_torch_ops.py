@@ -1,0 +1,50 @@
+"""The torch custom-op wrappers: fake (meta) shapes on CPU, and on the GPU
+the same results as the direct binding, inside torch.compile without a
+graph break (aot_eager backend: no code generation around the ops)."""
+
+import pytest
+import torch
+
+from flashattention_attention_attn_b200 import inputs
+import flashattention_attention_attn_b200.torch_ops  # noqa: F401  (registers torch.ops.fa_b200)
+
+
+def test_fake_shapes_without_running_anything():
+    from torch._subclasses.fake_tensor import FakeTensorMode
+    with FakeTensorMode():
+        q = torch.empty(2, 300, 32, 128, dtype=torch.bfloat16)
+        k = torch.empty(2, 400, 8, 128, dtype=torch.bfloat16)
+        o, lse = torch.ops.fa_b200.attn_fwd(q, k, k, True, 0.088)
+        assert o.shape == q.shape and o.dtype == torch.bfloat16
+        assert lse.shape == (2, 32, 300) and lse.dtype == torch.float32
+        qd = torch.empty(5, 32, 128, dtype=torch.bfloat16)
+        kc = torch.empty(40, 16, 8, 128, dtype=torch.bfloat16)
+        bt = torch.empty(5, 8, dtype=torch.int32)
+        od = torch.ops.fa_b200.paged_attn_decode(qd, kc, kc, bt, torch.empty(5, dtype=torch.int32), 0)
+        assert od.shape == qd.shape
+
+
+@pytest.mark.gpu
+def test_ops_match_binding_and_compile_without_graph_break():
+    import flashattention_attention_attn_b200 as fa
+    ps = inputs.PrefillSpec(B=1, Hq=8, Hkv=2, T=200, S=200, d=128, causal=True, seed=60)
+    q, k, v = [t.cuda() for t in inputs.make_prefill(ps)]
+    ds = inputs.DecodeSpec(B=3, Hq=32, Hkv=8, d=128, block_size=16, max_blocks=16, ctx_lo=10, ctx_hi=250, seed=61)
+    d = inputs.make_paged(ds)
+    dq, kc, vc, bt, sl = d.q.cuda(), d.k_cache.cuda(), d.v_cache.cuda(), d.block_table.cuda(), d.seq_lens.cuda()
+
+    o_ref = torch.empty_like(q)
+    lse_ref = torch.empty(1, 8, 200, device="cuda")
+    fa.attn_fwd(q, k, v, o_ref, lse_ref, 1, 8, 2, 200, 200, 128, True, ps.scale)
+    od_ref = torch.empty_like(dq)
+    fa.paged_attn_decode(dq, kc, vc, bt, sl, 3, 32, 8, 128, 16, 16, 0, od_ref)
+
+    def f(q, k, v, dq, kc, vc, bt, sl):
+        o, lse = torch.ops.fa_b200.attn_fwd(q, k, v, True, ps.scale)
+        od = torch.ops.fa_b200.paged_attn_decode(dq, kc, vc, bt, sl, 0)
+        return o, lse, od
+
+    g = torch.compile(f, backend="aot_eager", fullgraph=True)
+    o, lse, od = g(q, k, v, dq, kc, vc, bt, sl)
+    torch.cuda.synchronize()
+    assert torch.equal(o, o_ref) and torch.equal(lse, lse_ref) and torch.equal(od, od_ref)
