@@ -12,13 +12,15 @@ measured HBM bandwidth, and value = 100 * (sum over ranks of ideal time) /
 summed over the GPUs of the job.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                    [--workload step|long|varlen|chunked]
+                    [--workload step|long|varlen|chunked|fp8]
 
 `--workload long` times the long-context pair (T=S=16384 prefill and a
 131072-token split-KV decode) with the same accounting; `--workload varlen`
 replaces the prefill by 16 packed sequences of U[64, 2048] tokens
 (attn_fwd_varlen); `--workload chunked` by a 512-token chunk of each of 8
-sequences against their paged cache of 1k-8k tokens (paged_attn_prefill).  `--impl reference`
+sequences against their paged cache of 1k-8k tokens (paged_attn_prefill);
+`--workload fp8` keeps the step but stores the decode cache as FP8 e4m3
+(paged_attn_decode_fp8; decode bytes count 1 byte per cached element).  `--impl reference`
 times the fp64 CPU oracle (the only reference implementation there is) on a
 bounded sample of the same step.
 """
@@ -44,12 +46,21 @@ WORKLOAD_SETS = {
     "long": ("long_prefill_16k", "long_decode_131k"),
     "varlen": ("varlen_prefill_16seq", "paged_decode_b64"),
     "chunked": ("chunked_prefill_paged", "paged_decode_b64"),
+    "fp8": ("llama3_8b_prefill", "paged_decode_b64:fp8"),
 }
+
+
+def decode_workload(dname):
+    """(spec name, FP8 cache?) of a decode workload name ("name" or "name:fp8")."""
+    base, _, kind = dname.partition(":")
+    return base, kind == "fp8"
 
 
 class PrefillCase:
     """The prefill half of a step: dense (attn_fwd) or packed (attn_fwd_varlen); `--workload chunked` by a 512-token chunk of each of 8
-sequences against their paged cache of 1k-8k tokens (paged_attn_prefill)."""
+sequences against their paged cache of 1k-8k tokens (paged_attn_prefill);
+`--workload fp8` keeps the step but stores the decode cache as FP8 e4m3
+(paged_attn_decode_fp8; decode bytes count 1 byte per cached element)."""
 
     def __init__(self, name, seed, dev, fa, inputs, workloads):
         import torch
@@ -261,11 +272,17 @@ def cpu_baseline(pname, dname, peaks, seed_offset=0, budget_s=20.0):
         t_prefill, flops, pdesc = _cpu_prefill_chunked(pname, seed_offset, orc, inputs, workloads, f)
     else:
         t_prefill, flops, pdesc = _cpu_prefill_dense(pname, seed_offset, orc, inputs, workloads, f)
-    ds = inputs.WORKLOADS[dname]
-    dinp = inputs.make_paged(ds, seed=ds.seed + seed_offset)
+    dbase, dfp8 = decode_workload(dname)
+    ds = inputs.WORKLOADS[dbase]
+    if dfp8:
+        dinp = inputs.make_paged_fp8(ds, seed=ds.seed + seed_offset)
+        kc = dinp.k_scale * orc.decode_e4m3(dinp.k_cache.numpy())
+        vc = dinp.v_scale * orc.decode_e4m3(dinp.v_cache.numpy())
+    else:
+        dinp = inputs.make_paged(ds, seed=ds.seed + seed_offset)
+        kc, vc = f(dinp.k_cache), f(dinp.v_cache)
     # decode sample: leading sequences until ~budget/2 spent or 4 sequences
     lens = dinp.seq_lens.numpy()
-    kc, vc = f(dinp.k_cache), f(dinp.v_cache)
     qq = f(dinp.q)
     done_tok, td, nseq = 0, 0.0, 0
     for b in range(len(lens)):
@@ -277,7 +294,7 @@ def cpu_baseline(pname, dname, peaks, seed_offset=0, budget_s=20.0):
         if nseq >= 4 or td > budget_s / 2:
             break
     t_decode = td * float(lens.sum()) / max(done_tok, 1)
-    dbytes = workloads.decode_bytes(lens, ds.Hq, ds.Hkv, ds.d, ds.block_size)
+    dbytes = workloads.decode_bytes(lens, ds.Hq, ds.Hkv, ds.d, ds.block_size, kv_elem_bytes=1 if dfp8 else 2)
     ideal = flops / (peaks["bf16_tflops"] * 1e12) + dbytes / (peaks["hbm_gbs"] * 1e9)
     est = t_prefill + t_decode
     return {"value": 100.0 * ideal / est, "unit": UNIT, "cores": int(cores), "kind": "oracle",
@@ -317,12 +334,16 @@ def main():
     if fa.attn_check_support(local_rank) != 0:
         raise RuntimeError("device not supported by the library")
 
-    ds = inputs.WORKLOADS[dname]
+    dbase, dfp8 = decode_workload(dname)
+    ds = inputs.WORKLOADS[dbase]
     # weak scaling: every rank runs its own batch (different seeds), no exchange
     pspec = (inputs.VARLEN_WORKLOADS.get(pname) or inputs.CHUNKED_WORKLOADS.get(pname)
              or inputs.WORKLOADS[pname])
     pre = PrefillCase(pname, dist_util.rank_seed(pspec.seed, rank), dev, fa, inputs, workloads)
-    dinp = inputs.make_paged(ds, seed=dist_util.rank_seed(ds.seed, rank))
+    if dfp8:
+        dinp = inputs.make_paged_fp8(ds, seed=dist_util.rank_seed(ds.seed, rank))
+    else:
+        dinp = inputs.make_paged(ds, seed=dist_util.rank_seed(ds.seed, rank))
     qd_, kc, vc = dinp.q.to(dev), dinp.k_cache.to(dev), dinp.v_cache.to(dev)
     bt, sl = dinp.block_table.to(dev), dinp.seq_lens.to(dev)
     od = torch.empty(ds.B, ds.Hq, ds.d, device=dev, dtype=torch.bfloat16)
@@ -330,13 +351,21 @@ def main():
     stream = torch.cuda.current_stream(dev)
 
     flops = pre.flops
-    dbytes = workloads.decode_bytes(dinp.seq_lens.tolist(), ds.Hq, ds.Hkv, ds.d, ds.block_size)
+    dbytes = workloads.decode_bytes(dinp.seq_lens.tolist(), ds.Hq, ds.Hkv, ds.d, ds.block_size,
+                                    kv_elem_bytes=1 if dfp8 else 2)
     splits = args.num_splits
+
+    def decode_call():
+        if dfp8:
+            fa.paged_attn_decode_fp8(qd_, kc, vc, bt, sl, ds.B, ds.Hq, ds.Hkv, ds.d, ds.block_size, maxb, splits,
+                                     dinp.k_scale, dinp.v_scale, od, stream)
+        else:
+            fa.paged_attn_decode(qd_, kc, vc, bt, sl, ds.B, ds.Hq, ds.Hkv, ds.d, ds.block_size, maxb, splits, od,
+                                 stream)
 
     def step():
         pre.call(stream)
-        fa.paged_attn_decode(qd_, kc, vc, bt, sl, ds.B, ds.Hq, ds.Hkv, ds.d, ds.block_size, maxb, splits, od,
-                             stream)
+        decode_call()
 
     for _ in range(max(3, args.warmup)):
         step()
@@ -358,8 +387,7 @@ def main():
         ev[i][0].record(stream)
         pre.call(stream)
         ev[i][1].record(stream)
-        fa.paged_attn_decode(qd_, kc, vc, bt, sl, ds.B, ds.Hq, ds.Hkv, ds.d, ds.block_size, maxb, splits, od,
-                             stream)
+        decode_call()
         ev[i][2].record(stream)
     end.record(stream)
     torch.cuda.synchronize()
@@ -437,7 +465,8 @@ def main():
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K, "warmup": args.warmup,
         "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "bf16", "data": "synthetic (seeded N(0,1) bf16; random block-id permutations)",
-        "config": {"workload": f"{pname} + {dname}", "prefill": pre.config, "decode": vars_of(ds),
+        "config": {"workload": f"{pname} + {dname}", "prefill": pre.config,
+                   "decode": {**vars_of(ds), "kv_cache": "fp8 e4m3" if dfp8 else "bf16"},
                    "decode_num_splits": splits or "auto", "parallelism": f"replicas x{world} (no exchange)",
                    "l2": "inputs larger than L2 (decode KV cache %.0f MB per step)" % (dbytes / 1e6)},
         "parts": {"prefill": {"ms": t_pre, "tflops": pre_tflops, "frac": pre_tflops / peaks["bf16_tflops"],
@@ -481,7 +510,7 @@ def run_reference(args, pname, dname, peaks, peak_src, world):
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic (same seeds as ours)",
         "config": {"workload": f"{pname} + {dname}", "prefill": vars_of(inputs.VARLEN_WORKLOADS.get(pname) or inputs.CHUNKED_WORKLOADS.get(pname)
                                      or inputs.WORKLOADS[pname]),
-                   "decode": vars_of(inputs.WORKLOADS[dname])},
+                   "decode": vars_of(inputs.WORKLOADS[decode_workload(dname)[0]])},
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": info["cores"], "kind": "oracle",
                          "sample": info["sample"]},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},

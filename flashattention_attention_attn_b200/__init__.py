@@ -15,7 +15,7 @@ call does, and raises if it is missing.
 from . import inputs  # noqa: F401  (seeded synthetic inputs; no arithmetic)
 
 _BINDING_NAMES = {
-    "attn_fwd", "attn_fwd_varlen", "paged_attn_decode", "paged_attn_decode_noalloc", "paged_attn_prefill", "attn_check_support", "attn_status_string",
+    "attn_fwd", "attn_fwd_varlen", "paged_attn_decode", "paged_attn_decode_fp8", "paged_attn_decode_noalloc", "paged_attn_prefill", "attn_check_support", "attn_status_string",
     "attn_read_device_status", "attn_selftest_bounded_wait", "library", "library_path", "AttnError",
 }
 

@@ -46,6 +46,9 @@ def library() -> ctypes.CDLL:
         lib.paged_attn_decode.argtypes = [vp, vp, vp, vp, vp, c_int, c_int, c_int, c_int, c_int, c_int, c_int,
                                           vp, vp]
         lib.paged_attn_decode.restype = c_int
+        lib.paged_attn_decode_fp8.argtypes = [vp, vp, vp, vp, vp, c_int, c_int, c_int, c_int, c_int, c_int, c_int,
+                                              c_float, c_float, vp, vp]
+        lib.paged_attn_decode_fp8.restype = c_int
         lib.paged_attn_decode_noalloc.argtypes = lib.paged_attn_decode.argtypes
         lib.paged_attn_decode_noalloc.restype = c_int
         lib.attn_check_support.argtypes = [c_int]
@@ -121,6 +124,16 @@ def paged_attn_decode(q, k_cache, v_cache, block_table, seq_lens, B, Hq, Hkv, d,
                                      int(num_splits), _ptr(o), _stream(stream))
     if rc != ATTN_OK:
         raise AttnError(rc, "paged_attn_decode")
+
+
+def paged_attn_decode_fp8(q, k_cache, v_cache, block_table, seq_lens, B, Hq, Hkv, d, block_size, max_blocks,
+                          num_splits, k_scale, v_scale, o, stream=None) -> None:
+    """paged_attn_decode over an FP8 e4m3 cache with per-tensor scales (see attn.h)."""
+    rc = library().paged_attn_decode_fp8(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_table), _ptr(seq_lens),
+                                         int(B), int(Hq), int(Hkv), int(d), int(block_size), int(max_blocks),
+                                         int(num_splits), float(k_scale), float(v_scale), _ptr(o), _stream(stream))
+    if rc != ATTN_OK:
+        raise AttnError(rc, "paged_attn_decode_fp8")
 
 
 def paged_attn_decode_noalloc(q, k_cache, v_cache, block_table, seq_lens, B, Hq, Hkv, d, block_size,

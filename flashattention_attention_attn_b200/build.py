@@ -23,7 +23,7 @@ LIB_DIR = os.path.join(PKG_DIR, "_lib")
 LIB_PATH = os.path.join(LIB_DIR, "libattn_b200.so")
 
 SOURCES = ["attn_api.cu"]
-HEADERS = ["sm100_ptx.cuh", "prefill_sm100.cuh", "decode_paged.cuh"]
+HEADERS = ["sm100_ptx.cuh", "prefill_sm100.cuh", "decode_paged.cuh", "decode_paged_fp8.cuh"]
 
 
 def nvcc_path() -> str:

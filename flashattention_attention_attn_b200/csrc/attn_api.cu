@@ -13,6 +13,7 @@
 
 #include "attn.h"
 #include "decode_paged.cuh"
+#include "decode_paged_fp8.cuh"
 #include "prefill_sm100.cuh"
 #include "sm100_ptx.cuh"
 
@@ -101,6 +102,7 @@ int prepare_device(int dev, DeviceState* st) {
       {reinterpret_cast<const void*>(prefill::prefill_fwd_sm100<128, prefill::kPaged>), prefill::smem_bytes<128>()},
       {reinterpret_cast<const void*>(decode::paged_decode_split<64>), decode::smem_bytes<64>()},
       {reinterpret_cast<const void*>(decode::paged_decode_split<128>), decode::smem_bytes<128>()},
+      {reinterpret_cast<const void*>(decode::paged_decode_split_fp8), decode::smem_bytes_fp8()},
   };
   for (const auto& k : kernels)
     if (cudaFuncSetAttribute(k.fn, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(k.bytes)) !=
@@ -160,6 +162,20 @@ int make_map_pool(CUtensorMap* map, const void* base, int Hkv, int D) {
   cuuint32_t estr[2] = {1, 1};
   CUresult r = encode_tiled()(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides,
                               box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? ATTN_OK : ATTN_ERR_CUDA;
+}
+
+// 2-D map over an e4m3 pool seen as [tokens, Hkv * 128] bytes: box (128, 16),
+// one 128-byte swizzle row per head row.
+int make_map_pool_fp8(CUtensorMap* map, const void* base, int Hkv) {
+  constexpr cuuint64_t kTokens = (1ull << 31) - 16;
+  cuuint64_t dims[2] = {cuuint64_t(Hkv) * 128, kTokens};
+  cuuint64_t strides[1] = {cuuint64_t(Hkv) * 128};
+  cuuint32_t box[2] = {128, 16};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = encode_tiled()(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box,
+                              estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS ? ATTN_OK : ATTN_ERR_CUDA;
 }
@@ -372,10 +388,92 @@ int launch_decode(const void* q, const void* kc, const void* vc, const int32_t* 
   return rc;
 }
 
+// FP8 (e4m3) cache: the same split / combine structure, 128-dim heads.
+int launch_decode_fp8(const void* q, const void* kc, const void* vc, const int32_t* table, const int32_t* lens,
+                      int B, int Hq, int Hkv, int max_blocks, int num_splits, float k_scale, float v_scale, void* o,
+                      cudaStream_t stream, const DeviceState* st) {
+  constexpr int D = decode::kFp8D;
+  CUtensorMap mk, mv;
+  if (make_map_pool_fp8(&mk, kc, Hkv) || make_map_pool_fp8(&mv, vc, Hkv)) return ATTN_ERR_CUDA;
+  const int groups = (Hkv + decode::kKH - 1) / decode::kKH;
+  if (num_splits <= 0) num_splits = auto_splits(B, groups, max_blocks, st->sms);
+  if (num_splits > max_blocks) num_splits = max_blocks;
+  const int chunk = (max_blocks + num_splits - 1) / num_splits;
+  num_splits = (max_blocks + chunk - 1) / chunk;
+  if (num_splits > 65535 || groups > 65535 || B > 65535) return ATTN_ERR_UNSUPPORTED;
+  decode::Params p;
+  p.q = static_cast<const __nv_bfloat16*>(q);
+  p.block_table = table;
+  p.seq_lens = lens;
+  p.o = static_cast<__nv_bfloat16*>(o);
+  p.part_o = nullptr;
+  p.part_lse = nullptr;
+  p.B = B;
+  p.Hq = Hq;
+  p.Hkv = Hkv;
+  p.max_blocks = max_blocks;
+  p.num_splits = num_splits;
+  p.chunk = chunk;
+  p.scale_log2 = (1.0f / std::sqrt(static_cast<float>(D))) * k_scale * 1.4426950408889634f;
+  p.v_scale = v_scale;
+  void* ws = nullptr;
+  if (num_splits > 1) {
+    const size_t rows = static_cast<size_t>(num_splits) * B * Hq;
+    const size_t bytes = rows * D * sizeof(float) + rows * sizeof(float);
+    cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
+    if (cudaStreamIsCapturing(stream, &cap) != cudaSuccess) {
+      cudaGetLastError();
+      return ATTN_ERR_CUDA;
+    }
+    const cudaError_t ae = (cap == cudaStreamCaptureStatusActive)
+                               ? cudaMallocAsync(&ws, bytes, stream)
+                               : cudaMallocFromPoolAsync(&ws, bytes, st->pool, stream);
+    if (ae != cudaSuccess) {
+      cudaGetLastError();
+      return ATTN_ERR_CUDA;
+    }
+    p.part_o = static_cast<float*>(ws);
+    p.part_lse = p.part_o + rows * D;
+  }
+  dim3 grid(num_splits, groups, B);
+  decode::paged_decode_split_fp8<<<grid, (decode::kKH + 1) * 32, decode::smem_bytes_fp8(), stream>>>(mk, mv, p);
+  int rc = launch_status();
+  if (rc == ATTN_OK && num_splits > 1) rc = launch_combine<D>(p, lens, stream);
+  if (ws != nullptr) cudaFreeAsync(ws, stream);
+  return rc;
+}
+
 }  // namespace
 }  // namespace attn
 
 using namespace attn;
+
+extern "C" int paged_attn_decode_fp8(const void* q, const void* k_cache, const void* v_cache,
+                                     const int32_t* block_table, const int32_t* seq_lens, int B, int Hq, int Hkv,
+                                     int d, int block_size, int max_blocks, int num_splits, float k_scale,
+                                     float v_scale, void* o, attn_stream_t stream_) {
+  cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+  if (B < 0 || Hq <= 0 || Hkv <= 0 || d <= 0 || block_size <= 0) return ATTN_ERR_INVALID_ARG;
+  if (Hq % Hkv != 0) return ATTN_ERR_INVALID_ARG;
+  if (!(k_scale > 0.f) || !std::isfinite(k_scale) || !(v_scale > 0.f) || !std::isfinite(v_scale))
+    return ATTN_ERR_INVALID_ARG;
+  if (B == 0) return ATTN_OK;
+  if (max_blocks <= 0) return ATTN_ERR_INVALID_ARG;
+  if (q == nullptr || k_cache == nullptr || v_cache == nullptr || block_table == nullptr || seq_lens == nullptr ||
+      o == nullptr)
+    return ATTN_ERR_INVALID_ARG;
+  if (d != decode::kFp8D) return ATTN_ERR_UNSUPPORTED;
+  if (block_size != decode::kBlock) return ATTN_ERR_UNSUPPORTED;
+  if (Hq / Hkv > 8) return ATTN_ERR_UNSUPPORTED;
+  if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(o)) return ATTN_ERR_UNSUPPORTED;
+  if ((reinterpret_cast<uintptr_t>(block_table) & 3u) || (reinterpret_cast<uintptr_t>(seq_lens) & 3u))
+    return ATTN_ERR_UNSUPPORTED;
+  DeviceState* st = nullptr;
+  int rc = current_device_state(&st);
+  if (rc != ATTN_OK) return rc;
+  return launch_decode_fp8(q, k_cache, v_cache, block_table, seq_lens, B, Hq, Hkv, max_blocks, num_splits, k_scale,
+                           v_scale, o, stream, st);
+}
 
 extern "C" int attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq, int Hkv,
                         int T, int S, int d, int causal, float scale, attn_stream_t stream_) {

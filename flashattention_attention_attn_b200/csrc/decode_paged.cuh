@@ -66,7 +66,8 @@ struct Params {
   float* part_lse;             // [num_splits, B, Hq]
   int B, Hq, Hkv, max_blocks;
   int num_splits, chunk;       // chunk = blocks per split
-  float scale_log2;            // scale * log2(e)
+  float scale_log2;            // scale * log2(e) (FP8 path: scale * k_scale * log2(e))
+  float v_scale = 1.0f;        // FP8 path: V = v_scale * v_cache
 };
 
 // Byte address of token row t, 16-byte unit u of a 128-byte-swizzled chunk.

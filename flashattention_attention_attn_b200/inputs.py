@@ -285,3 +285,27 @@ def make_chunked(spec: ChunkedSpec, ctx_lens=None, q_lens=None, seed: int | None
     cu_q[1:] = torch.cumsum(torch.tensor(q_lens, dtype=torch.int64), 0).to(torch.int32)
     q = _randn_bf16(gen, (int(cu_q[-1]), s.Hq, s.d))
     return ChunkedInputs(q=q, cu_q=cu_q, cache=cache)
+
+
+@dataclass
+class PagedInputsFp8:
+    """A paged cache stored as FP8 e4m3 codes with one scale per tensor."""
+    q: torch.Tensor            # [B, Hq, d] bf16
+    k_cache: torch.Tensor      # [num_blocks, block_size, Hkv, d] uint8 (e4m3 codes)
+    v_cache: torch.Tensor      # same
+    block_table: torch.Tensor
+    seq_lens: torch.Tensor
+    block_size: int
+    k_scale: float
+    v_scale: float
+
+
+def make_paged_fp8(spec: DecodeSpec, seed: int | None = None, seq_lens=None, k_scale: float = 0.75,
+                   v_scale: float = 1.25) -> PagedInputsFp8:
+    """As make_paged (same draws), with the K and V pools rounded to e4m3
+    (round to nearest even, values N(0, 1) fit without saturation) and kept
+    as raw codes; the logical cache is k_scale * K and v_scale * V."""
+    p = make_paged(spec, seed=seed, seq_lens=seq_lens)
+    to8 = lambda t: t.to(torch.float32).to(torch.float8_e4m3fn).view(torch.uint8)  # noqa: E731
+    return PagedInputsFp8(q=p.q, k_cache=to8(p.k_cache), v_cache=to8(p.v_cache), block_table=p.block_table,
+                          seq_lens=p.seq_lens, block_size=p.block_size, k_scale=k_scale, v_scale=v_scale)

@@ -41,10 +41,11 @@ def prefill_min_bytes(B: int, Hq: int, Hkv: int, T: int, S: int, d: int) -> int:
     return 2 * d * (B * T * Hq * 2 + B * S * Hkv * 2) + 4 * B * Hq * T
 
 
-def decode_bytes(seq_lens, Hq: int, Hkv: int, d: int, block_size: int) -> int:
+def decode_bytes(seq_lens, Hq: int, Hkv: int, d: int, block_size: int, kv_elem_bytes: int = 2) -> int:
+    """kv_elem_bytes: 2 for a bf16 cache, 1 for an FP8 cache."""
     lens = [int(x) for x in seq_lens]
     B = len(lens)
-    kv = sum(lens) * Hkv * d * 2 * 2
+    kv = sum(lens) * Hkv * d * kv_elem_bytes * 2
     qo = 2 * B * Hq * d * 2
     table = sum(math.ceil(L / block_size) for L in lens) * 4 + B * 4
     return kv + qo + table

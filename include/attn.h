@@ -210,6 +210,25 @@ int paged_attn_prefill(const void* q, const void* k_cache, const void* v_cache,
                        void* o, float* lse, attn_stream_t stream);
 
 /*
+ * paged_attn_decode_fp8 - paged_attn_decode with the KV cache stored as FP8
+ * e4m3 (OCP e4m3fn: 1 sign, 4 exponent bits with bias 7, 3 mantissa bits),
+ * one scale per tensor: K = k_scale * k_cache, V = v_scale * v_cache.  Half
+ * the bytes per cached token of the bf16 cache.
+ *
+ *   k_cache, v_cache [num_blocks, block_size, Hkv, d] e4m3 bytes (16-byte
+ *   aligned); all other arguments and the result as paged_attn_decode.
+ *   The arithmetic is f16 x f16 -> fp32 on the tensor cores (e4m3 values are
+ *   exact in f16; q and P are rounded to f16).
+ *   Supported: d == 128; block_size == 16; 1 <= Hq/Hkv <= 8; sm_100.
+ *   Errors: as paged_attn_decode; ATTN_ERR_INVALID_ARG also for a scale that
+ *   is not finite and positive.
+ */
+int paged_attn_decode_fp8(const void* q, const void* k_cache, const void* v_cache,
+                          const int32_t* block_table, const int32_t* seq_lens,
+                          int B, int Hq, int Hkv, int d, int block_size, int max_blocks,
+                          int num_splits, float k_scale, float v_scale, void* o, attn_stream_t stream);
+
+/*
  * paged_attn_decode_noalloc - paged_attn_decode for callers that must not
  * allocate device memory during the call.
  *

@@ -2,6 +2,7 @@
 from .fp64_attention import (  # noqa: F401
     attention,
     attention_varlen,
+    decode_e4m3,
     gather_paged_kv,
     paged_decode,
     paged_prefill,

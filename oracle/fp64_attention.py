@@ -53,6 +53,7 @@ __all__ = [
     "gather_paged_kv",
     "paged_decode",
     "paged_prefill",
+    "decode_e4m3",
     "split_paged_decode",
 ]
 
@@ -221,6 +222,21 @@ def paged_prefill(q, k_cache, v_cache, block_table, seq_lens, cu_q, block_size: 
         O[q0:q1] = ob[0]
         LSE[:, q0:q1] = lb[0]
     return O, LSE
+
+
+def decode_e4m3(codes):
+    """Exact values of FP8 e4m3 codes (OCP "e4m3fn": sign bit, 4 exponent
+    bits with bias 7, 3 mantissa bits; exponent 0 is subnormal; the two codes
+    with all exponent and mantissa bits set are NaN; there is no infinity).
+    Used to state the FP8 KV cache in fp64: K = k_scale * decode_e4m3(k_cache).
+    """
+    c = np.asarray(codes, dtype=np.uint8).astype(np.int64)
+    sign = np.where(c & 0x80, -1.0, 1.0)
+    e = (c >> 3) & 0xF
+    m = (c & 0x7).astype(np.float64)
+    val = np.where(e == 0, np.ldexp(m / 8.0, -6), np.ldexp(1.0 + m / 8.0, e - 7))
+    val = np.where((e == 15) & (m == 7), np.nan, val)
+    return sign * val
 
 
 def split_paged_decode(q, k_cache, v_cache, block_table, seq_lens, block_size: int,

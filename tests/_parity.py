@@ -114,3 +114,24 @@ def oracle_chunked(inp, causal, scale):
     c = inp.cache
     return orc.paged_prefill(f64(inp.q), f64(c.k_cache), f64(c.v_cache), c.block_table.numpy(), c.seq_lens.numpy(),
                              inp.cu_q.numpy(), c.block_size, scale, causal)
+
+
+def run_decode_fp8(inp, num_splits=0):
+    import flashattention_attention_attn_b200 as fa
+    B, Hq, d = inp.q.shape
+    Hkv = inp.k_cache.shape[2]
+    o = torch.full((B, Hq, d), float("nan"), device="cuda", dtype=torch.bfloat16)
+    fa.paged_attn_decode_fp8(inp.q.cuda(), inp.k_cache.cuda(), inp.v_cache.cuda(), inp.block_table.cuda(),
+                             inp.seq_lens.cuda(), B, Hq, Hkv, d, inp.block_size, inp.block_table.shape[1],
+                             num_splits, inp.k_scale, inp.v_scale, o)
+    torch.cuda.synchronize()
+    assert fa.attn_read_device_status(clear=True) == 0
+    return o.cpu()
+
+
+def oracle_decode_fp8(inp):
+    d = inp.q.shape[-1]
+    K = inp.k_scale * orc.decode_e4m3(inp.k_cache.numpy())
+    V = inp.v_scale * orc.decode_e4m3(inp.v_cache.numpy())
+    return orc.paged_decode(f64(inp.q), K, V, inp.block_table.numpy(), inp.seq_lens.numpy(), inp.block_size,
+                            1.0 / np.sqrt(d))

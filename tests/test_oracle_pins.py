@@ -353,3 +353,14 @@ def test_paged_prefill_equals_contiguous_tail_rows():
         Of, Lf = orc.attention(Q, K, V, 0.3, True)
         np.testing.assert_allclose(O[cu_q[b]:cu_q[b + 1]], Of[0, c - t:], rtol=0, atol=1e-12)
         np.testing.assert_allclose(L[:, cu_q[b]:cu_q[b + 1]], Lf[0, :, c - t:], rtol=0, atol=1e-12)
+
+
+def test_e4m3_decoder_hand_values_and_torch():
+    # hand values from the format: 0x38 = 2^0, 0x7e = 448 (largest), 0x01 = 2^-9,
+    # 0x08 = 2^-6 (smallest normal), 0xb0 = -0.5, 0x7f = NaN
+    got = orc.decode_e4m3([0x38, 0x7E, 0x01, 0x08, 0xB0, 0x00, 0x80, 0x3C])
+    np.testing.assert_array_equal(got, [1.0, 448.0, 2.0 ** -9, 2.0 ** -6, -0.5, 0.0, -0.0, 1.5])
+    assert np.isnan(orc.decode_e4m3([0x7F, 0xFF])).all()
+    codes = np.arange(256, dtype=np.uint8)
+    ref = torch.from_numpy(codes).view(torch.float8_e4m3fn).to(torch.float64).numpy()
+    np.testing.assert_array_equal(orc.decode_e4m3(codes), ref)
