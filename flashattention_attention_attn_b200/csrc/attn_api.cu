@@ -166,18 +166,31 @@ int make_map_pool(CUtensorMap* map, const void* base, int Hkv, int D) {
   return r == CUDA_SUCCESS ? ATTN_OK : ATTN_ERR_CUDA;
 }
 
-// 2-D map over an e4m3 pool seen as [tokens, Hkv * 128] bytes: box (128, 16),
-// one 128-byte swizzle row per head row.
-int make_map_pool_fp8(CUtensorMap* map, const void* base, int Hkv) {
+// 3-D map over a paged pool for the decode kernels: dims (one 128-byte row
+// of a head, tokens, 128-byte rows of a token), i.e. the token stride is
+// listed before the smaller row stride, so that one box of
+// (row, 16 tokens, rows_per_group) lands in shared memory as
+// [row of the group][token][128 bytes] -- one copy per tensor and block.
+int make_map_pool_group(CUtensorMap* map, const void* base, CUtensorMapDataType dt, int elem_bytes,
+                        int rows_per_token, int rows_per_group) {
   constexpr cuuint64_t kTokens = (1ull << 31) - 16;
-  cuuint64_t dims[2] = {cuuint64_t(Hkv) * 128, kTokens};
-  cuuint64_t strides[1] = {cuuint64_t(Hkv) * 128};
-  cuuint32_t box[2] = {128, 16};
-  cuuint32_t estr[2] = {1, 1};
-  CUresult r = encode_tiled()(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box,
-                              estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+  const cuuint32_t row_elems = 128 / elem_bytes;
+  cuuint64_t dims[3] = {row_elems, kTokens, cuuint64_t(rows_per_token)};
+  cuuint64_t strides[2] = {cuuint64_t(rows_per_token) * 128, 128};
+  cuuint32_t box[3] = {row_elems, 16, cuuint32_t(rows_per_group)};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = encode_tiled()(map, dt, 3, const_cast<void*>(base), dims, strides, box, estr,
+                              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS ? ATTN_OK : ATTN_ERR_CUDA;
+}
+
+int make_map_decode_bf16(CUtensorMap* map, const void* base, int Hkv, int D) {
+  return make_map_pool_group(map, base, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, Hkv * D / 64, decode::kKH * D / 64);
+}
+
+int make_map_decode_fp8(CUtensorMap* map, const void* base, int Hkv) {
+  return make_map_pool_group(map, base, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, Hkv, decode::kKH);
 }
 
 int launch_status() {
@@ -336,7 +349,7 @@ int launch_decode(const void* q, const void* kc, const void* vc, const int32_t* 
                   int Hq, int Hkv, int max_blocks, int num_splits, void* o, cudaStream_t stream,
                   const DeviceState* st) {
   CUtensorMap mk, mv;
-  if (make_map_pool(&mk, kc, Hkv, D) || make_map_pool(&mv, vc, Hkv, D)) return ATTN_ERR_CUDA;
+  if (make_map_decode_bf16(&mk, kc, Hkv, D) || make_map_decode_bf16(&mv, vc, Hkv, D)) return ATTN_ERR_CUDA;
   const int groups = (Hkv + decode::kKH - 1) / decode::kKH;
   if (num_splits <= 0) num_splits = auto_splits(B, groups, max_blocks, st->sms);
   if (num_splits > max_blocks) num_splits = max_blocks;
@@ -394,7 +407,7 @@ int launch_decode_fp8(const void* q, const void* kc, const void* vc, const int32
                       cudaStream_t stream, const DeviceState* st) {
   constexpr int D = decode::kFp8D;
   CUtensorMap mk, mv;
-  if (make_map_pool_fp8(&mk, kc, Hkv) || make_map_pool_fp8(&mv, vc, Hkv)) return ATTN_ERR_CUDA;
+  if (make_map_decode_fp8(&mk, kc, Hkv) || make_map_decode_fp8(&mv, vc, Hkv)) return ATTN_ERR_CUDA;
   const int groups = (Hkv + decode::kKH - 1) / decode::kKH;
   if (num_splits <= 0) num_splits = auto_splits(B, groups, max_blocks, st->sms);
   if (num_splits > max_blocks) num_splits = max_blocks;
@@ -710,7 +723,7 @@ int launch_decode_noalloc(const void* q, const void* kc, const void* vc, const i
   const size_t rows = static_cast<size_t>(num_splits) * B * Hq;
   if (num_splits > 1 && rows * (D + 1) * sizeof(float) > ATTN_NOALLOC_SCRATCH_BYTES) return ATTN_ERR_UNSUPPORTED;
   CUtensorMap mk, mv;
-  if (make_map_pool(&mk, kc, Hkv, D) || make_map_pool(&mv, vc, Hkv, D)) return ATTN_ERR_CUDA;
+  if (make_map_decode_bf16(&mk, kc, Hkv, D) || make_map_decode_bf16(&mv, vc, Hkv, D)) return ATTN_ERR_CUDA;
 
   decode::Params p;
   p.q = static_cast<const __nv_bfloat16*>(q);

@@ -127,7 +127,6 @@ __global__ void __launch_bounds__((kKH + 1) * 32, 2)
     // Lane i holds block-table entry blk0 + w*32 + i of the current window;
     // lane 0 issues the loads.  Entries past the range are never read.
     const int32_t* row = p.block_table + static_cast<size_t>(b) * p.max_blocks + blk0;
-    const int x0 = hg * kKH * D;  // first column of this head group in a token row
     int issued = 0;
     bool ok = true;
     for (int w = 0; w < n && ok; w += 32) {
@@ -140,14 +139,11 @@ __global__ void __launch_bounds__((kKH + 1) * 32, 2)
         if (lane == 0) {
           ok = mbar_wait(&sm.empty[s], ((j / kStages) & 1) ^ 1, abort_flag);
           if (ok) {
-            mbar_arrive_expect_tx(&sm.full[s], 2 * kh_act * C::kHeadBytes);
-            const int y = phys * kBlock;
-            for (int hh = 0; hh < kh_act; ++hh)
-#pragma unroll
-              for (int c = 0; c < C::kChunks; ++c) {
-                tma_load_2d(sm.k[s][hh][c], &tmK, &sm.full[s], x0 + hh * D + c * 64, y);
-                tma_load_2d(sm.v[s][hh][c], &tmV, &sm.full[s], x0 + hh * D + c * 64, y);
-              }
+            // one copy per tensor: the 16 token rows of the group's kKH heads
+            // (heads past Hkv are zero-filled and still count as bytes)
+            mbar_arrive_expect_tx(&sm.full[s], 2 * kKH * C::kHeadBytes);
+            tma_load_3d(sm.k[s][0][0], &tmK, &sm.full[s], 0, phys * kBlock, hg * kKH * C::kChunks);
+            tma_load_3d(sm.v[s][0][0], &tmV, &sm.full[s], 0, phys * kBlock, hg * kKH * C::kChunks);
             issued = j + 1;
           }
         }

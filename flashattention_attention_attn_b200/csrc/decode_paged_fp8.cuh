@@ -15,11 +15,13 @@
 // dimension, and q is laid into the B fragment with the same permutation:
 // a dot product does not depend on the order of its terms.  q carries
 // scale * k_scale * log2(e), so the scores come out in the log2 domain.
-// Output: O[8 heads x d] = P V with P (transposed by movmatrix) as the A
-// operand and V as the B operand: ldmatrix.trans on the e4m3 tile gives
-// each lane two tokens x two columns; byte permutes split even and odd
-// columns, each converted to f16 pairs over the two tokens.  v_scale is
-// applied once at the end.
+// Output: O^T[d x 8 heads] += V^T P, with P (transposed by movmatrix) as the
+// B operand.  ldmatrix.trans on the e4m3 tile gives each lane two tokens x
+// two adjacent columns (2j, 2j+1); byte permutes split them into an f16 pair
+// over the two tokens for column 2j and one for column 2j+1, which become
+// the A-fragment rows j and j + 8: each 16-row output tile holds its 16
+// columns in the order (0, 2, .., 14, 1, 3, .., 15).  v_scale is applied
+// once at the end.
 #pragma once
 
 #include "decode_paged.cuh"
@@ -96,12 +98,11 @@ __global__ void __launch_bounds__((kKH + 1) * 32, 2)
         if (lane == 0) {
           ok = mbar_wait(&sm.empty[s], ((j / kFp8Stages) & 1) ^ 1, abort_flag);
           if (ok) {
-            mbar_arrive_expect_tx(&sm.full[s], 2 * kh_act * kFp8HeadBytes);
-            for (int hh = 0; hh < kh_act; ++hh) {
-              const int x = (hg * kKH + hh) * D;
-              tma_load_2d(sm.k[s][hh], &tmK, &sm.full[s], x, phys * kBlock);
-              tma_load_2d(sm.v[s][hh], &tmV, &sm.full[s], x, phys * kBlock);
-            }
+            // one copy per tensor: the 16 token rows of the group's kKH heads
+            // (heads past Hkv are zero-filled and still count as bytes)
+            mbar_arrive_expect_tx(&sm.full[s], 2 * kKH * kFp8HeadBytes);
+            tma_load_3d(sm.k[s][0], &tmK, &sm.full[s], 0, phys * kBlock, hg * kKH);
+            tma_load_3d(sm.v[s][0], &tmV, &sm.full[s], 0, phys * kBlock, hg * kKH);
             issued = j + 1;
           }
         }
@@ -145,11 +146,11 @@ __global__ void __launch_bounds__((kKH + 1) * 32, 2)
 
   float m0 = -INFINITY, m1 = -INFINITY;  // running max, heads 2*quad, 2*quad+1 (log2 domain)
   float l0 = 0.f, l1 = 0.f;
-  float acc[D / 16][2][4];  // O[g_row][16u + 4*quad + 2*c01 + parity] in acc[u][parity][c01]
+  // O^T tile u: acc[u][0] = O[2q][16u + 2j], acc[u][1] = O[2q+1][16u + 2j],
+  // acc[u][2] = O[2q][16u + 2j + 1], acc[u][3] = O[2q+1][16u + 2j + 1]; j = lane / 4
+  float acc[D / 16][4];
 #pragma unroll
-  for (int u = 0; u < D / 16; ++u)
-#pragma unroll
-    for (int e = 0; e < 2; ++e) acc[u][e][0] = acc[u][e][1] = acc[u][e][2] = acc[u][e][3] = 0.f;
+  for (int u = 0; u < D / 16; ++u) acc[u][0] = acc[u][1] = acc[u][2] = acc[u][3] = 0.f;
 
   const int t0 = lane >> 2, t1 = t0 + 8;
   const int lm_mat = lane >> 3, lm_row = lane & 7;
@@ -202,22 +203,18 @@ __global__ void __launch_bounds__((kKH + 1) * 32, 2)
     const float p10 = ex2_approx(sc[2] - mn0), p11 = ex2_approx(sc[3] - mn1);
     l0 = fmaf(l0, al0, p00 + p10);
     l1 = fmaf(l1, al1, p01 + p11);
-    // the O rows of this lane belong to head g_row: its factor sits in lane g_row / 2
-    const float ae = __shfl_sync(0xffffffffu, al0, g_row >> 1);
-    const float ao = __shfl_sync(0xffffffffu, al1, g_row >> 1);
-    const float al = (g_row & 1) ? ao : ae;
 #pragma unroll
-    for (int u = 0; u < D / 16; ++u)
-#pragma unroll
-      for (int e = 0; e < 2; ++e) {
-        acc[u][e][0] *= al;
-        acc[u][e][1] *= al;
-      }
-    // P[8 heads x 16 tokens] as the A operand (rows 8-15 are padding: zero)
-    const uint32_t pa0 = movmatrix_trans(pack_f16x2(p00, p01));
-    const uint32_t pa2 = movmatrix_trans(pack_f16x2(p10, p11));
+    for (int u = 0; u < D / 16; ++u) {
+      acc[u][0] *= al0;
+      acc[u][1] *= al1;
+      acc[u][2] *= al0;
+      acc[u][3] *= al1;
+    }
+    // P^T (tokens x heads, C layout) -> P as the k16 x n8 B operand
+    const uint32_t pb0 = movmatrix_trans(pack_f16x2(p00, p01));
+    const uint32_t pb1 = movmatrix_trans(pack_f16x2(p10, p11));
 
-    // ---- O[8 x d] += P V ----
+    // ---- O^T[d x 8] += V^T P ----
     const uint32_t vbase = smem_u32(sm.v[s][warp]);
 #pragma unroll
     for (int ux = 0; ux < D / 32; ++ux) {
@@ -230,10 +227,11 @@ __global__ void __launch_bounds__((kKH + 1) * 32, 2)
 #pragma unroll
       for (int h2 = 0; h2 < 2; ++h2) {
         const uint32_t lo = r[2 * h2], hi = r[2 * h2 + 1];
-        const uint32_t ev0 = e4m3x2_to_f16x2(prmt(lo, 0u, 0x20u)), ev1 = e4m3x2_to_f16x2(prmt(hi, 0u, 0x20u));
-        const uint32_t od0 = e4m3x2_to_f16x2(prmt(lo, 0u, 0x31u)), od1 = e4m3x2_to_f16x2(prmt(hi, 0u, 0x31u));
-        mma_f16_16816(acc[2 * ux + h2][0], pa0, 0u, pa2, 0u, ev0, ev1);
-        mma_f16_16816(acc[2 * ux + h2][1], pa0, 0u, pa2, 0u, od0, od1);
+        const uint32_t a0 = e4m3x2_to_f16x2(prmt(lo, 0u, 0x20u));  // column 2j, tokens 2q, 2q+1
+        const uint32_t a1 = e4m3x2_to_f16x2(prmt(lo, 0u, 0x31u));  // column 2j + 1
+        const uint32_t a2 = e4m3x2_to_f16x2(prmt(hi, 0u, 0x20u));  // column 2j, tokens 8 + ...
+        const uint32_t a3 = e4m3x2_to_f16x2(prmt(hi, 0u, 0x31u));
+        mma_f16_16816(acc[2 * ux + h2], a0, a1, a2, a3, pb0, pb1);
       }
     }
     __syncwarp();
@@ -246,34 +244,36 @@ __global__ void __launch_bounds__((kKH + 1) * 32, 2)
     l1 += __shfl_xor_sync(0xffffffffu, l1, off);
   }
   if (!ok) return;
-  // statistics of this lane's output head g_row
-  const float le = __shfl_sync(0xffffffffu, l0, g_row >> 1), lo_ = __shfl_sync(0xffffffffu, l1, g_row >> 1);
-  const float me = __shfl_sync(0xffffffffu, m0, g_row >> 1), mo = __shfl_sync(0xffffffffu, m1, g_row >> 1);
-  const float lg = (g_row & 1) ? lo_ : le;
-  const float mg = (g_row & 1) ? mo : me;
-  if (!real_row) return;
-  const float inv = p.v_scale / lg;
-  const size_t head = static_cast<size_t>(b) * p.Hq + hk * G + g_row;
+  const int g0 = 2 * quad, g1 = 2 * quad + 1;
+  const float inv0 = p.v_scale / l0, inv1 = p.v_scale / l1;
+  const int j2 = 2 * g_row;  // this lane's even column within each 16-column tile
+  const size_t head0 = static_cast<size_t>(b) * p.Hq + hk * G;
   if (p.num_splits == 1) {
-    __nv_bfloat16* out = p.o + head * D;
 #pragma unroll
-    for (int u = 0; u < D / 16; ++u)
-#pragma unroll
-      for (int c = 0; c < 2; ++c) {
-        const int dd = 16 * u + 4 * quad + 2 * c;  // columns dd (even part) and dd + 1 (odd part)
-        *reinterpret_cast<uint32_t*>(out + dd) = pack_bf16x2(acc[u][0][c] * inv, acc[u][1][c] * inv);
-      }
+    for (int u = 0; u < D / 16; ++u) {
+      if (g0 < G)
+        *reinterpret_cast<uint32_t*>(p.o + (head0 + g0) * D + 16 * u + j2) =
+            pack_bf16x2(acc[u][0] * inv0, acc[u][2] * inv0);
+      if (g1 < G)
+        *reinterpret_cast<uint32_t*>(p.o + (head0 + g1) * D + 16 * u + j2) =
+            pack_bf16x2(acc[u][1] * inv1, acc[u][3] * inv1);
+    }
   } else {
-    const size_t rowi = static_cast<size_t>(split) * p.B * p.Hq + head;
-    float* out = p.part_o + rowi * D;
+    const size_t base = static_cast<size_t>(split) * p.B * p.Hq + head0;
 #pragma unroll
-    for (int u = 0; u < D / 16; ++u)
-#pragma unroll
-      for (int c = 0; c < 2; ++c) {
-        const int dd = 16 * u + 4 * quad + 2 * c;
-        *reinterpret_cast<float2*>(out + dd) = make_float2(acc[u][0][c] * inv, acc[u][1][c] * inv);
-      }
-    if (quad == 0) p.part_lse[rowi] = (mg + __log2f(lg)) * 0.69314718055994531f;
+    for (int u = 0; u < D / 16; ++u) {
+      if (g0 < G)
+        *reinterpret_cast<float2*>(p.part_o + (base + g0) * D + 16 * u + j2) =
+            make_float2(acc[u][0] * inv0, acc[u][2] * inv0);
+      if (g1 < G)
+        *reinterpret_cast<float2*>(p.part_o + (base + g1) * D + 16 * u + j2) =
+            make_float2(acc[u][1] * inv1, acc[u][3] * inv1);
+    }
+    if (g_row == 0) {
+      constexpr float kLn2 = 0.69314718055994531f;
+      if (g0 < G) p.part_lse[base + g0] = (m0 + __log2f(l0)) * kLn2;
+      if (g1 < G) p.part_lse[base + g1] = (m1 + __log2f(l1)) * kLn2;
+    }
   }
 }
 
