@@ -29,6 +29,8 @@
 // sum always share the same reference, so the final O / l is unchanged.
 #pragma once
 
+#include <type_traits>
+
 #include "sm100_ptx.cuh"
 
 namespace attn {
@@ -202,7 +204,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int t = 0; t < 2; ++t) {
       mbar_init(&sm.q_full[t], 1);
       mbar_init(&sm.s_full[t], 1);
-      for (int c = 0; c < kPChunks; ++c) mbar_init(&sm.p_full[t][c], kBM);
+      for (int c = 0; c < kPChunks; ++c) mbar_init(&sm.p_full[t][c], 4);  // one arrive per softmax warp
       mbar_init(&sm.o_full[t], 1);
     }
     for (int s = 0; s < C::kStages; ++s) {
@@ -441,52 +443,66 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       const float mx = fmaxf(fmax3(fmax3(mx8[0], mx8[1], mx8[2]), fmax3(mx8[3], mx8[4], mx8[5]), mx8[6]), mx8[7]);
       const float m_new = fmaxf(m_used, mx * sl2);
-      if (m_new - m_used > kRescaleThreshold) {  // false while both are -inf (NaN)
-        if (m_used != -INFINITY) {
-          // O_t already holds P V of earlier tiles (their MMAs completed
-          // before this tile's S was committed): rescale it in place.
-          const float alpha = ex2_approx(m_used - m_new);
-          l *= alpha;
+      const bool move = m_new - m_used > kRescaleThreshold;  // false while both are -inf (NaN)
+      // O_t already holds P V of earlier tiles (their MMAs completed before
+      // this tile's S was committed) unless the row has seen no key yet.
+      const bool rescale = move && m_used != -INFINITY;
+      if (__any_sync(0xffffffffu, rescale)) {
+        // tcgen05.ld / st are warp-wide: the whole warp takes the round trip,
+        // rows that keep their reference with a factor of 1.
+        const float alpha = rescale ? ex2_approx(m_used - m_new) : 1.f;
+        l *= alpha;
 #pragma unroll
-          for (int c = 0; c < D / 32; ++c) {
-            uint32_t u[32];
-            tmem_ld32_sync(tO + c * 32, u);
+        for (int c = 0; c < D / 32; ++c) {
+          uint32_t u[32];
+          tmem_ld32_sync(tO + c * 32, u);
 #pragma unroll
-            for (int i = 0; i < 32; ++i) u[i] = __float_as_uint(__uint_as_float(u[i]) * alpha);
-            tmem_st_x32(tO + c * 32, u);
-          }
+          for (int i = 0; i < 32; ++i) u[i] = __float_as_uint(__uint_as_float(u[i]) * alpha);
+          tmem_st_x32(tO + c * 32, u);
         }
-        m_used = m_new;
       }
+      if (move) m_used = m_new;
       const float mref = (m_used == -INFINITY) ? 0.f : m_used;
-      const bool poly_ok = lim >= kBN;  // no masked score in this tile
-      (void)poly_ok;
-      // x = s * scale * log2(e) - m and the row sum in packed fp32 pairs.
+      // x = s * scale * log2(e) - m and the row sum in packed fp32 pairs;
+      // P = 2^x goes to tensor memory as bf16 pairs, chunk by chunk.
       const float2 c2 = make_float2(sl2, sl2);
       const float2 nm2 = make_float2(-mref, -mref);
       float2 sum4[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
                         make_float2(0.f, 0.f)};
+      auto exp_store = [&](auto poly_pairs) {
+        constexpr int kPoly = decltype(poly_pairs)::value;  // pairs of every 4 on the FMA pipe
 #pragma unroll
-      for (int c = 0; c < kBN / 32; ++c) {
-        uint32_t pk[16];
+        for (int c = 0; c < kBN / 32; ++c) {
+          uint32_t pk[16];
 #pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          const float2 x = __ffma2_rn(make_float2(s[c * 32 + 2 * i], s[c * 32 + 2 * i + 1]), c2, nm2);
-          float2 pp;
-          if ((i & 3) < kPolyPairsOf4 && poly_ok) {
-            pp = exp2_poly2(x);
-          } else {
-            pp = make_float2(ex2_approx(x.x), ex2_approx(x.y));
+          for (int i = 0; i < 16; ++i) {
+            const float2 x = __ffma2_rn(make_float2(s[c * 32 + 2 * i], s[c * 32 + 2 * i + 1]), c2, nm2);
+            float2 pp;
+            if constexpr (kPoly > 0) {
+              if ((i & 3) < kPoly) pp = exp2_poly2(x);
+              else pp = make_float2(ex2_approx(x.x), ex2_approx(x.y));
+            } else {
+              pp = make_float2(ex2_approx(x.x), ex2_approx(x.y));
+            }
+            sum4[i & 3] = __fadd2_rn(sum4[i & 3], pp);
+            pk[i] = pack_bf16x2(pp.x, pp.y);
           }
-          sum4[i & 3] = __fadd2_rn(sum4[i & 3], pp);
-          pk[i] = pack_bf16x2(pp.x, pp.y);
+          tmem_st_x16(tS + c * 16, pk);  // P overwrites the first 64 columns of S
+          if ((c + 1) % (4 / kPChunks) == 0) {
+            tmem_st_wait();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&sm.p_full[t][(c + 1) / (4 / kPChunks) - 1]);
+          }
         }
-        tmem_st_x16(tS + c * 16, pk);  // P overwrites the first 64 columns of S
-        if ((c + 1) % (4 / kPChunks) == 0) {
-          tmem_st_wait();
-          tc_fence_before();
-          mbar_arrive(&sm.p_full[t][(c + 1) / (4 / kPChunks) - 1]);
-        }
+      };
+      // The polynomial clamps its input, so it is only used where no score
+      // of the warp's rows is masked; the choice is warp-uniform because the
+      // tcgen05.st inside is a warp-wide (.sync.aligned) instruction.
+      if (kPolyPairsOf4 > 0 && __all_sync(0xffffffffu, lim >= kBN)) {
+        exp_store(std::integral_constant<int, kPolyPairsOf4>{});
+      } else {
+        exp_store(std::integral_constant<int, 0>{});
       }
       const float2 s01 = __fadd2_rn(sum4[0], sum4[1]);
       const float2 s23 = __fadd2_rn(sum4[2], sum4[3]);
