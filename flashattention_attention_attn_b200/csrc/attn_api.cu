@@ -198,12 +198,37 @@ int launch_status() {
   return e == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
 }
 
+// Launch as a programmatic dependent of the previous work on the stream: the
+// CTAs may be scheduled during the previous grid's tail and do their setup
+// there; every kernel launched this way calls grid_dependency_wait() before
+// its first global memory access.
+template <typename... KArgs, typename... Args>
+int launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
+               Args&&... args) {
+  cudaLaunchConfig_t cfg;
+  std::memset(&cfg, 0, sizeof(cfg));
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...) != cudaSuccess) {
+    cudaGetLastError();
+    return ATTN_ERR_CUDA;
+  }
+  return ATTN_OK;
+}
+
 template <int D>
 int launch_prefill(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq, int Hkv,
                    int T, int S, int causal, float scale, cudaStream_t stream) {
-  CUtensorMap mq, mk, mv, mo;
+  CUtensorMap mq, mk, mv;
   if (make_map_bthd(&mq, q, B, T, Hq, D) || make_map_bthd(&mk, k, B, S, Hkv, D) ||
-      make_map_bthd(&mv, v, B, S, Hkv, D) || make_map_bthd(&mo, o, B, T, Hq, D))
+      make_map_bthd(&mv, v, B, S, Hkv, D))
     return ATTN_ERR_CUDA;
   prefill::Params p;
   std::memset(&p, 0, sizeof(p));
@@ -219,9 +244,8 @@ int launch_prefill(const void* q, const void* k, const void* v, void* o, float* 
   p.num_mblocks = (T + 2 * prefill::kBM - 1) / (2 * prefill::kBM);
   const long long grid = static_cast<long long>(p.num_mblocks) * Hq * B;
   if (grid > 0x7fffffffLL) return ATTN_ERR_UNSUPPORTED;
-  prefill::prefill_fwd_sm100<D, prefill::kDense><<<static_cast<unsigned>(grid), prefill::kThreads,
-                                         prefill::smem_bytes<D>(), stream>>>(mq, mk, mv, mo, p);
-  return launch_status();
+  return launch_pdl(prefill::prefill_fwd_sm100<D, prefill::kDense>, dim3(static_cast<unsigned>(grid)),
+                    dim3(prefill::kThreads), prefill::smem_bytes<D>(), stream, mq, mk, mv, p);
 }
 
 // Packed sequences: the maps see [total, H, D] as one batch; the grid covers
@@ -231,9 +255,9 @@ template <int D>
 int launch_prefill_varlen(const void* q, const void* k, const void* v, void* o, float* lse, const int32_t* cu_q,
                           const int32_t* cu_k, int B, int max_q, int total_q, int total_k, int Hq, int Hkv,
                           int causal, float scale, cudaStream_t stream) {
-  CUtensorMap mq, mk, mv, mo;
+  CUtensorMap mq, mk, mv;
   if (make_map_bthd(&mq, q, 1, total_q, Hq, D) || make_map_bthd(&mk, k, 1, total_k, Hkv, D) ||
-      make_map_bthd(&mv, v, 1, total_k, Hkv, D) || make_map_bthd(&mo, o, 1, total_q, Hq, D))
+      make_map_bthd(&mv, v, 1, total_k, Hkv, D))
     return ATTN_ERR_CUDA;
   prefill::Params p;
   std::memset(&p, 0, sizeof(p));
@@ -252,9 +276,8 @@ int launch_prefill_varlen(const void* q, const void* k, const void* v, void* o, 
   p.num_mblocks = (max_q + 2 * prefill::kBM - 1) / (2 * prefill::kBM);
   const long long grid = static_cast<long long>(p.num_mblocks) * Hq * B;
   if (grid > 0x7fffffffLL) return ATTN_ERR_UNSUPPORTED;
-  prefill::prefill_fwd_sm100<D, prefill::kVarlen><<<static_cast<unsigned>(grid), prefill::kThreads,
-                                        prefill::smem_bytes<D>(), stream>>>(mq, mk, mv, mo, p);
-  return launch_status();
+  return launch_pdl(prefill::prefill_fwd_sm100<D, prefill::kVarlen>, dim3(static_cast<unsigned>(grid)),
+                    dim3(prefill::kThreads), prefill::smem_bytes<D>(), stream, mq, mk, mv, p);
 }
 
 // Chunked prefill against the paged cache: packed queries as in varlen,
@@ -263,9 +286,8 @@ template <int D>
 int launch_prefill_paged(const void* q, const void* kc, const void* vc, const int32_t* table, const int32_t* lens,
                          const int32_t* cu_q, void* o, float* lse, int B, int max_q, int total_q, int Hq, int Hkv,
                          int max_blocks, int causal, float scale, cudaStream_t stream) {
-  CUtensorMap mq, mk, mv, mo;
-  if (make_map_bthd(&mq, q, 1, total_q, Hq, D) || make_map_pool(&mk, kc, Hkv, D) || make_map_pool(&mv, vc, Hkv, D) ||
-      make_map_bthd(&mo, o, 1, total_q, Hq, D))
+  CUtensorMap mq, mk, mv;
+  if (make_map_bthd(&mq, q, 1, total_q, Hq, D) || make_map_pool(&mk, kc, Hkv, D) || make_map_pool(&mv, vc, Hkv, D))
     return ATTN_ERR_CUDA;
   prefill::Params p;
   std::memset(&p, 0, sizeof(p));
@@ -285,9 +307,8 @@ int launch_prefill_paged(const void* q, const void* kc, const void* vc, const in
   p.num_mblocks = (max_q + 2 * prefill::kBM - 1) / (2 * prefill::kBM);
   const long long grid = static_cast<long long>(p.num_mblocks) * Hq * B;
   if (grid > 0x7fffffffLL) return ATTN_ERR_UNSUPPORTED;
-  prefill::prefill_fwd_sm100<D, prefill::kPaged><<<static_cast<unsigned>(grid), prefill::kThreads,
-                                                   prefill::smem_bytes<D>(), stream>>>(mq, mk, mv, mo, p);
-  return launch_status();
+  return launch_pdl(prefill::prefill_fwd_sm100<D, prefill::kPaged>, dim3(static_cast<unsigned>(grid)),
+                    dim3(prefill::kThreads), prefill::smem_bytes<D>(), stream, mq, mk, mv, p);
 }
 
 // Splits for num_splits <= 0.  The host does not know the sequence lengths
@@ -394,8 +415,8 @@ int launch_decode(const void* q, const void* kc, const void* vc, const int32_t* 
     p.part_lse = p.part_o + rows * D;
   }
   dim3 grid(num_splits, groups, B);
-  decode::paged_decode_split<D><<<grid, (decode::kKH + 1) * 32, decode::smem_bytes<D>(), stream>>>(mk, mv, p);
-  int rc = launch_status();
+  int rc = launch_pdl(decode::paged_decode_split<D>, grid, dim3((decode::kKH + 1) * 32), decode::smem_bytes<D>(),
+                      stream, mk, mv, p);
   if (rc == ATTN_OK && num_splits > 1) rc = launch_combine<D>(p, lens, stream);
   if (ws != nullptr) cudaFreeAsync(ws, stream);
   return rc;
@@ -449,8 +470,8 @@ int launch_decode_fp8(const void* q, const void* kc, const void* vc, const int32
     p.part_lse = p.part_o + rows * D;
   }
   dim3 grid(num_splits, groups, B);
-  decode::paged_decode_split_fp8<<<grid, (decode::kKH + 1) * 32, decode::smem_bytes_fp8(), stream>>>(mk, mv, p);
-  int rc = launch_status();
+  int rc = launch_pdl(decode::paged_decode_split_fp8, grid, dim3((decode::kKH + 1) * 32), decode::smem_bytes_fp8(),
+                      stream, mk, mv, p);
   if (rc == ATTN_OK && num_splits > 1) rc = launch_combine<D>(p, lens, stream);
   if (ws != nullptr) cudaFreeAsync(ws, stream);
   return rc;

@@ -83,15 +83,27 @@ __global__ void __launch_bounds__((kKH + 1) * 32, 2)
   extern __shared__ uint8_t smem_raw[];
   Smem<D>& sm = *reinterpret_cast<Smem<D>*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
 
-  // Let the combine kernel (launched as a programmatic dependent) be
-  // scheduled once every CTA of this grid has started; it waits for this
-  // grid's completion before it reads any partial.
-  asm volatile("griddepcontrol.launch_dependents;");
   const int split = blockIdx.x;
   const int hg = blockIdx.y;  // kv-head group
   const int b = blockIdx.z;
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
+  const int kh_act = min(kKH, p.Hkv - hg * kKH);  // kv heads of this group that exist
+
+  // Barrier setup overlaps the previous grid's tail (programmatic launch);
+  // global memory is read only after grid_dependency_wait().  Then the
+  // combine kernel (this grid's programmatic dependent) may be scheduled; it
+  // waits for this grid's completion before it reads any partial.
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(&sm.full[s], 1);
+      mbar_init(&sm.empty[s], kh_act);
+    }
+    sm.abort_flag = 0;
+    fence_mbarrier_init();
+  }
+  grid_dependency_wait();
+  grid_launch_dependents();
 
   const int L = p.seq_lens[b];
   const int nb = (L + kBlock - 1) / kBlock;
@@ -109,16 +121,6 @@ __global__ void __launch_bounds__((kKH + 1) * 32, 2)
     return;
   }
   const int n = blk1 - blk0;
-  const int kh_act = min(kKH, p.Hkv - hg * kKH);  // kv heads of this group that exist
-
-  if (threadIdx.x == 0) {
-    for (int s = 0; s < kStages; ++s) {
-      mbar_init(&sm.full[s], 1);
-      mbar_init(&sm.empty[s], kh_act);
-    }
-    sm.abort_flag = 0;
-    fence_mbarrier_init();
-  }
   __syncthreads();
   volatile int* abort_flag = &sm.abort_flag;
 
@@ -327,7 +329,7 @@ __global__ void __launch_bounds__((kKH + 1) * 32, 2)
 // max pass) and kUnroll rows in flight per lane; lane c owns D/32
 // consecutive columns.  The row's warps are merged in shared memory in a
 // fixed order (deterministic).  Launched as a programmatic dependent of the
-// split kernel: everything before griddepcontrol.wait overlaps its tail.
+// split kernel: everything before grid_dependency_wait() overlaps its tail.
 template <int WPR>
 struct CombineShape {
   static constexpr int kWarps = WPR > 8 ? WPR : 8;
@@ -352,12 +354,13 @@ __global__ void __launch_bounds__(CombineShape<WPR>::kWarps * 32)
   __shared__ float s_acc[Shape::kWarps][D];
   __shared__ float s_m[Shape::kWarps], s_w[Shape::kWarps];
 
+  grid_dependency_wait();
+  grid_launch_dependents();
   int nsp = 0;
   if (live) {
-    const int L = seq_lens[row_id / Hq];  // an input of the call, not written by the split kernel
+    const int L = seq_lens[row_id / Hq];
     nsp = min(num_splits, (((L + kBlock - 1) / kBlock) + chunk - 1) / chunk);  // splits holding data
   }
-  asm volatile("griddepcontrol.wait;" ::: "memory");
   const size_t stride = static_cast<size_t>(B) * Hq;  // rows between splits
 
   float m = -INFINITY, wsum = 0.f;  // log2-domain running max and weight sum

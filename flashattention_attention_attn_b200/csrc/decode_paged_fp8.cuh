@@ -49,13 +49,26 @@ __global__ void __launch_bounds__((kKH + 1) * 32, 2)
   constexpr int D = kFp8D;
   extern __shared__ uint8_t smem_raw[];
   SmemFp8& sm = *reinterpret_cast<SmemFp8*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  asm volatile("griddepcontrol.launch_dependents;");
-
   const int split = blockIdx.x;
   const int hg = blockIdx.y;
   const int b = blockIdx.z;
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
+  const int kh_act = min(kKH, p.Hkv - hg * kKH);
+
+  // As in the bf16 kernel: barrier setup before the wait for the previous
+  // grid, global reads after it, then the combine may be scheduled.
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kFp8Stages; ++s) {
+      mbar_init(&sm.full[s], 1);
+      mbar_init(&sm.empty[s], kh_act);
+    }
+    sm.abort_flag = 0;
+    fence_mbarrier_init();
+  }
+  grid_dependency_wait();
+  grid_launch_dependents();
+
   const int L = p.seq_lens[b];
   const int nb = (L + kBlock - 1) / kBlock;
   const int blk0 = split * p.chunk;
@@ -70,16 +83,6 @@ __global__ void __launch_bounds__((kKH + 1) * 32, 2)
     return;
   }
   const int n = blk1 - blk0;
-  const int kh_act = min(kKH, p.Hkv - hg * kKH);
-
-  if (threadIdx.x == 0) {
-    for (int s = 0; s < kFp8Stages; ++s) {
-      mbar_init(&sm.full[s], 1);
-      mbar_init(&sm.empty[s], kh_act);
-    }
-    sm.abort_flag = 0;
-    fence_mbarrier_init();
-  }
   __syncthreads();
   volatile int* abort_flag = &sm.abort_flag;
 

@@ -164,8 +164,7 @@ __device__ __forceinline__ int kv_tiles_for(int r0, int T, int S, int causal) {
 template <int D, int MODE>
 __global__ void __launch_bounds__(kThreads, 1)
     prefill_fwd_sm100(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
-                      const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
-                      const Params p) {
+                      const __grid_constant__ CUtensorMap tmV, const Params p) {
   using C = Config<D>;
   extern __shared__ uint8_t smem_raw[];
   Smem<D>& sm = *reinterpret_cast<Smem<D>*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -183,24 +182,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int hk = h / (p.Hq / p.Hkv);
   const int m0 = mb * 2 * kBM;
   constexpr bool VARLEN = MODE != kDense;  // packed queries and outputs
-  int T = p.T, S = p.S, qoff = 0, koff = 0, bc = b;  // bc: batch coordinate of the maps
-  if constexpr (VARLEN) {
-    qoff = p.cu_q[b];
-    T = p.cu_q[b + 1] - qoff;
-    if constexpr (MODE == kPaged) {
-      S = p.seq_lens[b];
-    } else {
-      koff = p.cu_k[b];
-      S = p.cu_k[b + 1] - koff;
-    }
-    bc = 0;
-    if (m0 >= T) return;  // this query block lies past the sequence (uniform over the CTA)
-  }
-  const int n0 = kv_tiles_for(m0, T, S, p.causal);
-  const int n1 = kv_tiles_for(m0 + kBM, T, S, p.causal);
-  const int n_max = max(n0, n1);
 
-  if (threadIdx.x == 0) {
+  // Setup that reads no global memory (barriers, tensor memory, descriptor
+  // prefetch) overlaps the tail of the previous grid on the stream; this
+  // kernel is launched as its programmatic dependent.
+  if (warp == kWarpLoad && lane == 0) {
     for (int t = 0; t < 2; ++t) {
       mbar_init(&sm.q_full[t], 1);
       mbar_init(&sm.s_full[t], 1);
@@ -217,10 +203,62 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(&sm.v_tail, 1);
     sm.abort_flag = 0;
     fence_mbarrier_init();
+    tma_prefetch_desc(&tmQ);
+    tma_prefetch_desc(&tmK);
+    tma_prefetch_desc(&tmV);
   }
   if (warp == 0) {
     tmem_alloc(&sm.tmem_base, kTmemCols);
     tmem_relinquish();
+  }
+  grid_dependency_wait();
+  grid_launch_dependents();
+
+  int T = p.T, S = p.S, qoff = 0, koff = 0, bc = b;  // bc: batch coordinate of the maps
+  if constexpr (VARLEN) {
+    qoff = p.cu_q[b];
+    T = p.cu_q[b + 1] - qoff;
+    if constexpr (MODE == kPaged) {
+      S = p.seq_lens[b];
+    } else {
+      koff = p.cu_k[b];
+      S = p.cu_k[b + 1] - koff;
+    }
+    bc = 0;
+    if (m0 >= T) {
+      // This query block lies past the sequence (uniform over the CTA).
+      if (warp == 0) {
+        tc_fence_before();
+        __syncwarp();
+        tc_fence_after();
+        tmem_dealloc(sm.tmem_base, kTmemCols);
+      }
+      return;
+    }
+  }
+  const int n0 = kv_tiles_for(m0, T, S, p.causal);
+  const int n1 = kv_tiles_for(m0 + kBM, T, S, p.causal);
+  const int n_max = max(n0, n1);
+
+  // The first copies leave before the CTA-wide barrier: Q of both tiles and,
+  // for contiguous keys, K / V tile 0 (paged tiles need the warp's table reads).
+  const int pre = (MODE != kPaged && n_max > 0) ? 1 : 0;  // K / V tiles issued here
+  if (warp == kWarpLoad && lane == 0) {
+    const int nt[2] = {n0, n1};
+    for (int t = 0; t < 2; ++t) {
+      if (nt[t] == 0) continue;
+      mbar_arrive_expect_tx(&sm.q_full[t], C::kTileBytes);
+      for (int c = 0; c < C::kChunks; ++c)
+        tma_load_4d(sm.q[t][c], &tmQ, &sm.q_full[t], c * 64, h, qoff + m0 + t * kBM, bc);
+    }
+    if constexpr (MODE != kPaged) {
+      if (pre) {
+        mbar_arrive_expect_tx(&sm.k_full[0], C::kTileBytes);
+        for (int c = 0; c < C::kChunks; ++c) tma_load_4d(sm.k[0][c], &tmK, &sm.k_full[0], c * 64, hk, koff, bc);
+        mbar_arrive_expect_tx(&sm.v_full[0], C::kTileBytes);
+        for (int c = 0; c < C::kChunks; ++c) tma_load_4d(sm.v[0][c], &tmV, &sm.v_full[0], c * 64, hk, koff, bc);
+      }
+    }
   }
   tc_fence_before();
   __syncthreads();
@@ -232,23 +270,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ------------------------------ producer ------------------------------
     // The whole warp runs the loop (paged mode loads block ids in parallel);
     // lane 0 waits on the barriers and issues the copies.
-    if (lane == 0) {
-      tma_prefetch_desc(&tmQ);
-      tma_prefetch_desc(&tmK);
-      tma_prefetch_desc(&tmV);
-    }
     const int nt[2] = {n0, n1};
-    if (lane == 0) {
-      for (int t = 0; t < 2; ++t) {
-        if (nt[t] == 0) continue;
-        mbar_arrive_expect_tx(&sm.q_full[t], C::kTileBytes);
-        for (int c = 0; c < C::kChunks; ++c)
-          tma_load_4d(sm.q[t][c], &tmQ, &sm.q_full[t], c * 64, h, qoff + m0 + t * kBM, bc);
-      }
-    }
-    int k_issued = 0, v_issued = 0;  // K / V tiles whose loads were issued
+    int k_issued = pre, v_issued = pre;  // K / V tiles whose loads were issued
     bool tail_issued = false;
-    for (int j = 0; j < n_max; ++j) {
+    for (int j = pre; j < n_max; ++j) {
       const int s = j % C::kStages;
       const uint32_t ph = (j / C::kStages) & 1;
       int nblk = kBN / 16;   // 16-token blocks loaded into this tile
@@ -444,24 +469,26 @@ __global__ void __launch_bounds__(kThreads, 1)
       const float mx = fmaxf(fmax3(fmax3(mx8[0], mx8[1], mx8[2]), fmax3(mx8[3], mx8[4], mx8[5]), mx8[6]), mx8[7]);
       const float m_new = fmaxf(m_used, mx * sl2);
       const bool move = m_new - m_used > kRescaleThreshold;  // false while both are -inf (NaN)
-      // O_t already holds P V of earlier tiles (their MMAs completed before
-      // this tile's S was committed) unless the row has seen no key yet.
-      const bool rescale = move && m_used != -INFINITY;
-      if (__any_sync(0xffffffffu, rescale)) {
-        // tcgen05.ld / st are warp-wide: the whole warp takes the round trip,
-        // rows that keep their reference with a factor of 1.
-        const float alpha = rescale ? ex2_approx(m_used - m_new) : 1.f;
-        l *= alpha;
+      if (__any_sync(0xffffffffu, move)) {
+        // O_t already holds P V of earlier tiles (their MMAs completed before
+        // this tile's S was committed) unless the row has seen no key yet.
+        const bool rescale = move && m_used != -INFINITY;
+        if (__any_sync(0xffffffffu, rescale)) {
+          // tcgen05.ld / st are warp-wide: the whole warp takes the round
+          // trip, rows that keep their reference with a factor of 1.
+          const float alpha = rescale ? ex2_approx(m_used - m_new) : 1.f;
+          l *= alpha;
 #pragma unroll
-        for (int c = 0; c < D / 32; ++c) {
-          uint32_t u[32];
-          tmem_ld32_sync(tO + c * 32, u);
+          for (int c = 0; c < D / 32; ++c) {
+            uint32_t u[32];
+            tmem_ld32_sync(tO + c * 32, u);
 #pragma unroll
-          for (int i = 0; i < 32; ++i) u[i] = __float_as_uint(__uint_as_float(u[i]) * alpha);
-          tmem_st_x32(tO + c * 32, u);
+            for (int i = 0; i < 32; ++i) u[i] = __float_as_uint(__uint_as_float(u[i]) * alpha);
+            tmem_st_x32(tO + c * 32, u);
+          }
         }
+        if (move) m_used = m_new;
       }
-      if (move) m_used = m_new;
       const float mref = (m_used == -INFINITY) ? 0.f : m_used;
       // x = s * scale * log2(e) - m and the row sum in packed fp32 pairs;
       // P = 2^x goes to tensor memory as bf16 pairs, chunk by chunk.
@@ -514,11 +541,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       ok = __all_sync(0xffffffffu, mbar_wait(&sm.o_full[t], (nt - 1) & 1, abort_flag));
       tc_fence_after();
     }
-    // Epilogue: O / l -> bf16, staged (128-byte swizzled) in this tile's Q
-    // buffer, then one TMA store per 64-wide chunk (rows >= T are clipped).
+    // Epilogue: O / l -> bf16, each thread storing its own row (256 B for
+    // D = 128) straight from registers; rows past the sequence end are not
+    // stored.  No staging and no wait: the CTA can retire at once.
     const float inv_l = (l > 0.f) ? 1.0f / l : 0.f;
-    const bool have_o = ok && nt > 0;
-    uint8_t* stage = reinterpret_cast<uint8_t*>(sm.q[t][0]);
+    const bool have_o = ok && nt > 0;  // warp-uniform: tcgen05.ld is warp-wide
+    const size_t orow = VARLEN ? static_cast<size_t>(qoff) + row : static_cast<size_t>(b) * T + row;
+    uint4* dst = reinterpret_cast<uint4*>(p.o + (orow * p.Hq + h) * D);
 #pragma unroll
     for (int c = 0; c < D / 32; ++c) {
       uint32_t u[32];
@@ -532,37 +561,16 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
       for (int i = 0; i < 16; ++i)
         pk[i] = pack_bf16x2(__uint_as_float(u[2 * i]) * inv_l, __uint_as_float(u[2 * i + 1]) * inv_l);
-      uint8_t* chunk = stage + (c / 2) * C::kChunkBytes + r * 128;
+      if (row < T) {
 #pragma unroll
-      for (int q4 = 0; q4 < 4; ++q4) {
-        const int unit = (c & 1) * 4 + q4;  // 16-byte unit within the 128-byte row
-        *reinterpret_cast<uint4*>(chunk + ((unit ^ (r & 7)) << 4)) =
-            make_uint4(pk[4 * q4], pk[4 * q4 + 1], pk[4 * q4 + 2], pk[4 * q4 + 3]);
+        for (int q4 = 0; q4 < 4; ++q4)
+          dst[c * 4 + q4] = make_uint4(pk[4 * q4], pk[4 * q4 + 1], pk[4 * q4 + 2], pk[4 * q4 + 3]);
       }
     }
     if (p.lse != nullptr && row < T) {
       const float lse = (l > 0.f) ? (m_used + __log2f(l)) * 0.69314718055994531f : -INFINITY;
       const size_t lse_rows = VARLEN ? static_cast<size_t>(p.total_q) : static_cast<size_t>(T);
       p.lse[(static_cast<size_t>(bc) * p.Hq + h) * lse_rows + qoff + row] = lse;
-    }
-    fence_proxy_async_smem();
-    named_barrier_sync(1 + t, kBM);
-    const int r0 = m0 + t * kBM;
-    if (VARLEN && r0 + kBM > T) {
-      // The tile crosses the end of the sequence: a 128-row store would
-      // overwrite the next sequence's rows, so each thread stores its own row.
-      if (row < T) {
-        uint8_t* dst = reinterpret_cast<uint8_t*>(p.o) + ((static_cast<size_t>(qoff) + row) * p.Hq + h) * D * 2;
-#pragma unroll
-        for (int u = 0; u < D / 8; ++u) {
-          const uint8_t* src = stage + (u / 8) * C::kChunkBytes + r * 128 + (((u & 7) ^ (r & 7)) << 4);
-          *reinterpret_cast<uint4*>(dst + u * 16) = *reinterpret_cast<const uint4*>(src);
-        }
-      }
-    } else if (r == 0 && r0 < T) {
-      for (int c = 0; c < C::kChunks; ++c) tma_store_4d(&tmO, stage + c * C::kChunkBytes, c * 64, h, qoff + r0, bc);
-      tma_store_commit();
-      tma_store_wait_read0();
     }
   }
 

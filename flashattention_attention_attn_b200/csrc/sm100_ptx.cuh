@@ -107,6 +107,17 @@ __device__ __forceinline__ void named_barrier_sync(uint32_t id, uint32_t nthread
 
 // ---------------------------------- TMA ------------------------------------
 // All loads are plain (no .multicast::cluster): every CTA fetches its own tiles.
+// ------------------------ programmatic dependent launch ----------------------
+// A kernel launched with programmatic stream serialization may start while
+// the previous grid on the stream is still running.  It must not touch global
+// memory before grid_dependency_wait(), which returns once that grid has
+// completed and its writes are visible (at once when there is none).
+__device__ __forceinline__ void grid_dependency_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
+// Lets the next grid on the stream be scheduled (it still waits for this one
+// to complete before it reads anything).
+__device__ __forceinline__ void grid_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap* map) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
 }
