@@ -52,6 +52,20 @@ WORKLOAD_SETS = {
 }
 
 
+# DRAM bytes (read + write) per launch of the dominant kernel of each step,
+# from the one-pass ncu launch lists of the same command (`dram__bytes_read.sum`
+# + `dram__bytes_write.sum`, mean over the captured launches), summarised in
+# profiles/launches_<workload>.md.  A value is dropped (None) whenever the
+# kernel changes after its capture.
+#   step / fp8: decode split kernel + LSE combine of one paged_attn_decode call
+#   long:       the attn_fwd launch
+TRAFFIC_BYTES = {
+    "step": 597.37e6 + 4.66e6 + 6.30e6,   # profiles/launches_llama3_8b_prefill_paged_decode_b64.md
+    "fp8": 298.98e6 + 3.43e6 + 6.30e6,    # profiles/launches_llama3_8b_prefill_paged_decode_b64_fp8.md
+    "long": 354.05e6 + 97.52e6,           # profiles/launches_long_prefill_16k_long_decode_131k.md
+}
+
+
 def decode_workload(dname):
     """(spec name, FP8 cache?) of a decode workload name ("name" or "name:fp8")."""
     base, _, kind = dname.partition(":")
@@ -77,6 +91,7 @@ sequences against their paged cache of 1k-8k tokens (paged_attn_prefill);
             lens_q = (ci.cu_q[1:] - ci.cu_q[:-1]).tolist()
             ctx = c.seq_lens.tolist()
             self.flops = sum(workloads.prefill_flops(1, sp.Hq, t, s_, sp.d, sp.causal) for t, s_ in zip(lens_q, ctx))
+            self.min_bytes = sum(workloads.prefill_min_bytes(1, sp.Hq, sp.Hkv, t, s_, sp.d) for t, s_ in zip(lens_q, ctx))
             self.max_q, self.total_q, self.max_blocks = ci.max_q, int(ci.cu_q[-1]), c.block_table.shape[1]
             self.dev_in = [t.to(dev) for t in self.host_in]
             self.o = torch.empty_like(self.dev_in[0])
@@ -89,6 +104,8 @@ sequences against their paged cache of 1k-8k tokens (paged_attn_prefill);
             lens_q = (vin.cu_q[1:] - vin.cu_q[:-1]).tolist()
             lens_k = (vin.cu_k[1:] - vin.cu_k[:-1]).tolist()
             self.flops = sum(workloads.prefill_flops(1, sp.Hq, t, s_, sp.d, sp.causal) for t, s_ in zip(lens_q, lens_k))
+            self.min_bytes = sum(workloads.prefill_min_bytes(1, sp.Hq, sp.Hkv, t, s_, sp.d)
+                                 for t, s_ in zip(lens_q, lens_k))
             self.max_q, self.total_q, self.total_k = vin.max_q, int(vin.cu_q[-1]), int(vin.cu_k[-1])
             self.dev_in = [t.to(dev) for t in self.host_in]
             self.o = torch.empty_like(self.dev_in[0])
@@ -99,6 +116,7 @@ sequences against their paged cache of 1k-8k tokens (paged_attn_prefill);
             q, k, v = inputs.make_prefill(sp, seed=seed)
             self.host_in = [q, k, v]
             self.flops = workloads.prefill_flops(sp.B, sp.Hq, sp.T, sp.S, sp.d, sp.causal)
+            self.min_bytes = workloads.prefill_min_bytes(sp.B, sp.Hq, sp.Hkv, sp.T, sp.S, sp.d)
             self.dev_in = [t.to(dev) for t in self.host_in]
             self.o = torch.empty_like(self.dev_in[0])
             self.lse = torch.empty(sp.B, sp.Hq, sp.T, device=dev, dtype=torch.float32)
@@ -134,7 +152,7 @@ def load_peaks():
 def parse_args():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--steps", type=int, default=2000)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", choices=sorted(WORKLOAD_SETS), default="step")
@@ -148,26 +166,54 @@ def parse_args():
 # clocks during the timed region (NVML reads only; nothing is changed)
 # --------------------------------------------------------------------------
 class ClockSampler:
+    """Samples SM clock and clock-event reasons every 20 ms from an
+    `nvidia-smi -lms` child process (independent of this process's GIL), with
+    NVML polling in a thread as the fallback.  Each sample is stamped with
+    time.perf_counter() when it arrives."""
     REASONS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
                0x8: "hw_slowdown", 0x10: "sync_boost", 0x20: "sw_thermal_slowdown",
                0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown", 0x100: "display_clock_setting"}
 
-    def __init__(self, device_index: int, period_s: float = 0.01):
+    def __init__(self, device_index: int, period_s: float = 0.02):
         self.samples = []
         self.period = period_s
+        # nvidia-smi and NVML number GPUs physically; CUDA_VISIBLE_DEVICES may
+        # not, so the device is named by its UUID when torch reports one.
+        self.ident = str(device_index)
+        try:
+            import torch
+            uuid = str(torch.cuda.get_device_properties(device_index).uuid)
+            if uuid:
+                self.ident = uuid if uuid.startswith("GPU-") else "GPU-" + uuid
+        except Exception:
+            pass
         self._stop = threading.Event()
         self._thr = None
+        self._proc = None
         self.max_mhz = None
+        self.source = None
+        self._nv = None
         try:
             import pynvml
             pynvml.nvmlInit()
             self._nv = pynvml
-            self._h = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self._h = (pynvml.nvmlDeviceGetHandleByUUID(self.ident.encode()) if self.ident.startswith("GPU-")
+                       else pynvml.nvmlDeviceGetHandleByIndex(device_index))
             self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
         except Exception:
             self._nv = None
 
-    def _run(self):
+    def _read_smi(self):
+        for line in self._proc.stdout:
+            parts = [x.strip() for x in line.split(",")]
+            try:
+                self.samples.append((time.perf_counter(), int(parts[0]), int(parts[2], 16)))
+                if self.max_mhz is None:
+                    self.max_mhz = int(parts[1])
+            except (ValueError, IndexError):
+                pass
+
+    def _poll_nvml(self):
         nv = self._nv
         while not self._stop.is_set():
             try:
@@ -178,19 +224,43 @@ class ClockSampler:
                 pass
             time.sleep(self.period)
 
-    def start(self):
-        if self._nv is not None:
-            self._thr = threading.Thread(target=self._run, daemon=True)
+    def start(self, wait_s: float = 5.0):
+        import shutil
+        import subprocess
+        smi = shutil.which("nvidia-smi")
+        if smi is not None:
+            try:
+                self._proc = subprocess.Popen(
+                    [smi, "-i", self.ident, "--query-gpu=clocks.sm,clocks.max.sm,clocks_event_reasons.active",
+                     "--format=csv,noheader,nounits", "-lms", str(int(self.period * 1000))],
+                    stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True, bufsize=1)
+                self._thr = threading.Thread(target=self._read_smi, daemon=True)
+                self.source = "nvidia-smi -lms %d" % int(self.period * 1000)
+            except OSError:
+                self._proc = None
+        if self._proc is None and self._nv is not None:
+            self._thr = threading.Thread(target=self._poll_nvml, daemon=True)
+            self.source = "nvml polling"
+        if self._thr is not None:
             self._thr.start()
+            t_end = time.perf_counter() + wait_s  # the timed region starts once samples flow
+            while not self.samples and time.perf_counter() < t_end:
+                time.sleep(0.01)
 
     def stop(self):
         self._stop.set()
+        if self._proc is not None:
+            self._proc.terminate()
+            try:
+                self._proc.wait(timeout=5)
+            except Exception:
+                self._proc.kill()
         if self._thr is not None:
-            self._thr.join()
+            self._thr.join(timeout=5)
 
     def summary(self, t0, t1):
-        if self._nv is None:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvml unavailable"], "samples": 0}
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": ["no clock samples"], "samples": 0}
         inside = [s for s in self.samples if t0 <= s[0] <= t1]
         use = inside or self.samples
         mhz = sorted(s[1] for s in use)
@@ -199,7 +269,8 @@ class ClockSampler:
             bits |= int(s[2])
         reasons = [name for bit, name in self.REASONS.items() if bits & bit and name != "gpu_idle"]
         return {"sm_mhz": mhz[len(mhz) // 2] if mhz else None, "sm_max_mhz": self.max_mhz,
-                "reasons": reasons, "samples": len(inside), "samples_total": len(self.samples)}
+                "reasons": reasons, "samples": len(inside), "samples_total": len(self.samples),
+                "source": self.source}
 
 
 # --------------------------------------------------------------------------
@@ -463,12 +534,15 @@ def main():
     dominant = "decode" if t_dec >= t_pre else "prefill"
     if dominant == "decode":
         roofline = {"bound": "hbm", "achieved": dec_gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                    "frac": dec_gbs / peaks["hbm_gbs"], "traffic": None,
+                    "frac": dec_gbs / peaks["hbm_gbs"], "traffic": TRAFFIC_BYTES.get(args.workload),
+                    "traffic_unit": "bytes per call (ncu DRAM read + write)", "algorithmic_bytes": dbytes,
                     "kernel": "paged_attn_decode (split kernel + LSE combine)",
                     "peak_source": f"{peak_src} (hbm_gbs)", "duration": PART_TIMING}
     else:
         roofline = {"bound": "tensor", "achieved": pre_tflops, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
-                    "frac": pre_tflops / peaks["bf16_tflops"], "traffic": None, "kernel": "attn_fwd",
+                    "frac": pre_tflops / peaks["bf16_tflops"], "traffic": TRAFFIC_BYTES.get(args.workload),
+                    "traffic_unit": "bytes per launch (ncu DRAM read + write)", "algorithmic_bytes": pre.min_bytes,
+                    "kernel": "attn_fwd",
                     "peak_source": f"{peak_src} (bf16_tflops, burst)", "duration": PART_TIMING}
     launches_per_step = 1 + 1 + 1  # prefill, decode split kernel, LSE combine
     line = {

@@ -313,11 +313,12 @@ int launch_prefill_paged(const void* q, const void* kc, const void* vc, const in
 
 // Splits for num_splits <= 0.  The host does not know the sequence lengths
 // (they are on the device), so the choice assumes every sequence fills
-// max_blocks: a single sequence is cut into one wave of equal units (two
-// decode CTAs fit on an SM); a batch into about four waves, so that the
-// scheduler can balance units of unequal length.  At least 8 blocks per unit.
-int auto_splits(int B, int groups, int max_blocks, int sms) {
-  const long long slots = 2LL * sms;
+// max_blocks: a single sequence is cut into one wave of equal units
+// (ctas_per_sm decode CTAs fit on an SM); a batch into about four waves, so
+// that the scheduler can balance units of unequal length.  At least 8 blocks
+// per unit.
+int auto_splits(int B, int groups, int max_blocks, int sms, int ctas_per_sm = 2) {
+  const long long slots = static_cast<long long>(ctas_per_sm) * sms;
   const long long waves = (B == 1) ? 1 : 4;
   const long long blocks = static_cast<long long>(B) * groups * max_blocks;
   long long chunk = (blocks + waves * slots - 1) / (waves * slots);
@@ -430,7 +431,7 @@ int launch_decode_fp8(const void* q, const void* kc, const void* vc, const int32
   CUtensorMap mk, mv;
   if (make_map_decode_fp8(&mk, kc, Hkv) || make_map_decode_fp8(&mv, vc, Hkv)) return ATTN_ERR_CUDA;
   const int groups = (Hkv + decode::kKH - 1) / decode::kKH;
-  if (num_splits <= 0) num_splits = auto_splits(B, groups, max_blocks, st->sms);
+  if (num_splits <= 0) num_splits = auto_splits(B, groups, max_blocks, st->sms, decode::kFp8CtasPerSm);
   if (num_splits > max_blocks) num_splits = max_blocks;
   const int chunk = (max_blocks + num_splits - 1) / num_splits;
   num_splits = (max_blocks + chunk - 1) / chunk;
