@@ -314,12 +314,14 @@ int launch_prefill_paged(const void* q, const void* kc, const void* vc, const in
 // Splits for num_splits <= 0.  The host does not know the sequence lengths
 // (they are on the device), so the choice assumes every sequence fills
 // max_blocks: a single sequence is cut into one wave of equal units
-// (ctas_per_sm decode CTAs fit on an SM); a batch into about four waves, so
-// that the scheduler can balance units of unequal length.  At least 8 blocks
-// per unit.
+// (ctas_per_sm decode CTAs fit on an SM); a batch into about three waves, so
+// that the scheduler can balance units of unequal length.  (A sweep on a
+// batch of 64 sequences of 256-4096 tokens put three waves -- 7 splits --
+// ahead of four -- 10 splits -- for both caches, and two far behind.)  At
+// least 8 blocks per unit.
 int auto_splits(int B, int groups, int max_blocks, int sms, int ctas_per_sm = 2) {
   const long long slots = static_cast<long long>(ctas_per_sm) * sms;
-  const long long waves = (B == 1) ? 1 : 4;
+  const long long waves = (B == 1) ? 1 : 3;
   const long long blocks = static_cast<long long>(B) * groups * max_blocks;
   long long chunk = (blocks + waves * slots - 1) / (waves * slots);
   if (chunk < 8) chunk = 8;

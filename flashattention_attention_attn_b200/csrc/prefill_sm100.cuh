@@ -206,6 +206,19 @@ __global__ void __launch_bounds__(kThreads, 1)
     tma_prefetch_desc(&tmQ);
     tma_prefetch_desc(&tmK);
     tma_prefetch_desc(&tmV);
+    if constexpr (MODE == kDense) {
+      // The first tiles into L2 while the previous grid finishes (the
+      // shapes are known without reading memory in this mode).
+      if (kv_tiles_for(m0, p.T, p.S, p.causal) + kv_tiles_for(m0 + kBM, p.T, p.S, p.causal) > 0) {
+        for (int t = 0; t < 2; ++t)
+          if (m0 + t * kBM < p.T)
+            for (int c = 0; c < C::kChunks; ++c) tma_prefetch_l2_4d(&tmQ, c * 64, h, m0 + t * kBM, b);
+        for (int c = 0; c < C::kChunks; ++c) {
+          tma_prefetch_l2_4d(&tmK, c * 64, hk, 0, b);
+          tma_prefetch_l2_4d(&tmV, c * 64, hk, 0, b);
+        }
+      }
+    }
   }
   if (warp == 0) {
     tmem_alloc(&sm.tmem_base, kTmemCols);
