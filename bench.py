@@ -60,9 +60,9 @@ WORKLOAD_SETS = {
 #   step / fp8: decode split kernel + LSE combine of one paged_attn_decode call
 #   long:       the attn_fwd launch
 TRAFFIC_BYTES = {
-    "step": 597.37e6 + 4.66e6 + 6.30e6,   # profiles/launches_llama3_8b_prefill_paged_decode_b64.md
-    "fp8": 298.98e6 + 3.43e6 + 6.30e6,    # profiles/launches_llama3_8b_prefill_paged_decode_b64_fp8.md
-    "long": 354.05e6 + 97.52e6,           # profiles/launches_long_prefill_16k_long_decode_131k.md
+    "step": 597.39e6 + 3.07e6 + 4.58e6,   # profiles/launches_llama3_8b_prefill_paged_decode_b64.md
+    "fp8": 299.01e6 + 2.57e6 + 4.58e6,    # profiles/launches_llama3_8b_prefill_paged_decode_b64_fp8.md
+    "long": 365.06e6 + 97.73e6,           # profiles/launches_long_prefill_16k_long_decode_131k.md
 }
 
 
