@@ -220,7 +220,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
   }
-  if (warp == 0) {
+  if (!VARLEN && warp == 0) {
     tmem_alloc(&sm.tmem_base, kTmemCols);
     tmem_relinquish();
   }
@@ -238,15 +238,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       S = p.cu_k[b + 1] - koff;
     }
     bc = 0;
-    if (m0 >= T) {
-      // This query block lies past the sequence (uniform over the CTA).
-      if (warp == 0) {
-        tc_fence_before();
-        __syncwarp();
-        tc_fence_after();
-        tmem_dealloc(sm.tmem_base, kTmemCols);
-      }
-      return;
+    // A query block past the sequence (uniform over the CTA) leaves before
+    // it allocates tensor memory: packed batches of short sequences have many.
+    if (m0 >= T) return;
+    if (warp == 0) {
+      tmem_alloc(&sm.tmem_base, kTmemCols);
+      tmem_relinquish();
     }
   }
   const int n0 = kv_tiles_for(m0, T, S, p.causal);
@@ -554,30 +551,53 @@ __global__ void __launch_bounds__(kThreads, 1)
       ok = __all_sync(0xffffffffu, mbar_wait(&sm.o_full[t], (nt - 1) & 1, abort_flag));
       tc_fence_after();
     }
-    // Epilogue: O / l -> bf16, each thread storing its own row (256 B for
-    // D = 128) straight from registers; rows past the sequence end are not
-    // stored.  No staging and no wait: the CTA can retire at once.
-    const float inv_l = (l > 0.f) ? 1.0f / l : 0.f;
-    const bool have_o = ok && nt > 0;  // warp-uniform: tcgen05.ld is warp-wide
-    const size_t orow = VARLEN ? static_cast<size_t>(qoff) + row : static_cast<size_t>(b) * T + row;
-    uint4* dst = reinterpret_cast<uint4*>(p.o + (orow * p.Hq + h) * D);
+    // Epilogue: O / l -> bf16.  Each warp stages its 32 rows in this tile's
+    // Q buffer (free: the tile's last QK^T completed before o_full fired),
+    // 16-byte chunks XOR-swizzled by row so that neither the row-wise writes
+    // nor the chunk-wise reads conflict on banks, then copies them out with
+    // whole rows per group of lanes (coalesced), skipping rows past the end.
+    // No wait on any copy: the CTA can retire at once.
+    {
+      constexpr int kRowBytes = D * 2;
+      constexpr int kChunksPerRow = kRowBytes / 16;  // 16 (D = 128) or 8 (D = 64)
+      constexpr int kRowsPerPass = 32 / kChunksPerRow;
+      const float inv_l = (l > 0.f) ? 1.0f / l : 0.f;
+      const bool have_o = ok && nt > 0;  // warp-uniform: tcgen05.ld is warp-wide
+      uint8_t* stage = reinterpret_cast<uint8_t*>(sm.q[t][0]) + (warp & 3) * 32 * kRowBytes;
+      uint8_t* my_row = stage + lane * kRowBytes;
 #pragma unroll
-    for (int c = 0; c < D / 32; ++c) {
-      uint32_t u[32];
-      if (have_o) {
-        tmem_ld32_sync(tO + c * 32, u);
-      } else {
+      for (int c = 0; c < D / 32; ++c) {
+        uint32_t u[32];
+        if (have_o) {
+          tmem_ld32_sync(tO + c * 32, u);
+        } else {
 #pragma unroll
-        for (int i = 0; i < 32; ++i) u[i] = 0u;
+          for (int i = 0; i < 32; ++i) u[i] = 0u;
+        }
+        uint32_t pk[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i)
+          pk[i] = pack_bf16x2(__uint_as_float(u[2 * i]) * inv_l, __uint_as_float(u[2 * i + 1]) * inv_l);
+#pragma unroll
+        for (int q4 = 0; q4 < 4; ++q4) {
+          const int chunk = (c * 4 + q4) ^ (lane & (kChunksPerRow - 1));
+          *reinterpret_cast<uint4*>(my_row + chunk * 16) =
+              make_uint4(pk[4 * q4], pk[4 * q4 + 1], pk[4 * q4 + 2], pk[4 * q4 + 3]);
+        }
       }
-      uint32_t pk[16];
-#pragma unroll
-      for (int i = 0; i < 16; ++i)
-        pk[i] = pack_bf16x2(__uint_as_float(u[2 * i]) * inv_l, __uint_as_float(u[2 * i + 1]) * inv_l);
-      if (row < T) {
-#pragma unroll
-        for (int q4 = 0; q4 < 4; ++q4)
-          dst[c * 4 + q4] = make_uint4(pk[4 * q4], pk[4 * q4 + 1], pk[4 * q4 + 2], pk[4 * q4 + 3]);
+      __syncwarp();
+      const int warp_row0 = t * kBM + (warp & 3) * 32;  // first row of this warp within the CTA's block
+      const int chunk = lane % kChunksPerRow;
+#pragma unroll 4
+      for (int pass = 0; pass < 32 / kRowsPerPass; ++pass) {
+        const int rl = pass * kRowsPerPass + lane / kChunksPerRow;  // row within the warp's 32
+        const int rrow = m0 + warp_row0 + rl;                       // row within the sequence
+        const uint4 val =
+            *reinterpret_cast<const uint4*>(stage + rl * kRowBytes + ((chunk ^ (rl & (kChunksPerRow - 1))) * 16));
+        if (rrow < T) {
+          const size_t orow = VARLEN ? static_cast<size_t>(qoff) + rrow : static_cast<size_t>(b) * T + rrow;
+          reinterpret_cast<uint4*>(p.o + (orow * p.Hq + h) * D)[chunk] = val;
+        }
       }
     }
     if (p.lse != nullptr && row < T) {
