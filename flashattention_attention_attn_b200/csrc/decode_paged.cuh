@@ -343,7 +343,7 @@ __global__ void __launch_bounds__(CombineShape<WPR>::kWarps * 32)
                 int num_splits, int chunk) {
   using Shape = CombineShape<WPR>;
   constexpr int kPer = D / 32;
-  constexpr int kUnroll = 4;
+  constexpr int kUnroll = (WPR == 1) ? 8 : 4;  // rows in flight per lane: one round for up to 8 splits
   constexpr float kLog2e = 1.4426950408889634f;
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
