@@ -13,7 +13,8 @@
 //   warps 0..KH-1  consumers, one kv head each, all G = Hq/Hkv query heads of
 //                  that kv head at once (the group shares every K/V load)
 //   warp  KH       producer: reads the block-table entries of the range and
-//                  issues one TMA load per 64-wide d chunk per head (K and V)
+//                  issues one TMA load per tensor per block (a 3-D view of
+//                  the pool brings the 16 token rows of all KH heads at once)
 // Per block, a consumer warp computes S^T[16 tokens x 8] = K q^T with
 // mma.sync m16n8k16 (query heads padded to 8), updates the running max / sum
 // of its heads, transposes P^T into the B-operand layout with movmatrix and

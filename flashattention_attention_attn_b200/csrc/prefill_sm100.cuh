@@ -20,6 +20,11 @@
 //   O_0 [256, 256+D), O_1 [256+D, 256+2D): fp32 output accumulators.
 // The two query tiles ping-pong: while the softmax warps of one tile work,
 // the tensor core runs the other tile's MMAs.
+// The kernel is launched as a programmatic dependent of the previous grid on
+// the stream: barrier set-up, the tensor-memory allocation and (dense mode) L2
+// prefetches of the first tiles happen before the grid-dependency wait.  The
+// epilogue stages each warp's 32 output rows in the tile's (by then free) Q
+// buffer and stores them coalesced.
 //
 // Softmax statistics are kept in the log2 domain (s * scale * log2 e) and the
 // exponentials use ex2.  The row max used as reference is only moved (and O
