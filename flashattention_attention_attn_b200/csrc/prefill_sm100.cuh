@@ -380,10 +380,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int t = 0; t < 2 && ok; ++t)
         if (nt[t] > 0) ok = mbar_wait(&sm.q_full[t], 0, abort_flag);
 
-      // O_t += P_t(jj) V(jj)
-      auto issue_pv = [&](int t, int jj) -> bool {
+      // O_t += P_t(jj) V(jj).  Every commit and every wait costs this thread
+      // ~100 cycles on the critical path of a P hand-off, so V(jj) is waited
+      // for once per iteration (wait_v: the tile that comes first) and O_t
+      // is committed only after the tile's last P V (last).
+      auto issue_pv = [&](int t, int jj, bool wait_v, bool last) -> bool {
         const int s = jj % C::kStages;
-        if (!mbar_wait(&sm.v_full[s], (jj / C::kStages) & 1, abort_flag)) return false;
+        if (wait_v && !mbar_wait(&sm.v_full[s], (jj / C::kStages) & 1, abort_flag)) return false;
         const uint32_t tS = tmem + t * kBN;
         const uint32_t tO = tmem + 2 * kBN + t * D;
         const uint32_t vbase = smem_u32(sm.v[s][0]);
@@ -401,7 +404,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             umma_ts(tO, tS + kk * 8, bdesc, idesc_pv, (jj > 0 || kk > 0) ? 1u : 0u);
           }
         }
-        umma_commit(&sm.o_full[t]);
+        if (last) umma_commit(&sm.o_full[t]);
         return true;
       };
 
@@ -411,7 +414,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_after();
         for (int t = 0; t < 2 && ok; ++t) {
           // the previous P_t must be consumed before S_t is overwritten
-          if (j >= 1 && j - 1 < nt[t]) ok = issue_pv(t, j - 1);
+          if (j >= 1 && j - 1 < nt[t]) ok = issue_pv(t, j - 1, t == 0 || j - 1 >= nt[0], j == nt[t]);
           if (ok && j < nt[t]) {
             const uint32_t tS = tmem + t * kBN;
             const uint32_t qbase = smem_u32(sm.q[t][0]);
@@ -433,7 +436,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (ok && n_max > 0) {
         const int jl = n_max - 1;
         for (int t = 0; t < 2 && ok; ++t)
-          if (jl < nt[t]) ok = issue_pv(t, jl);
+          if (jl < nt[t]) ok = issue_pv(t, jl, t == 0 || jl >= nt[0], true);
         if (ok) umma_commit(&sm.v_empty[jl % C::kStages]);
       }
       // Every MMA issued above is complete once mma_done fires; after an
@@ -553,7 +556,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
 
     if (ok && nt > 0) {
-      ok = __all_sync(0xffffffffu, mbar_wait(&sm.o_full[t], (nt - 1) & 1, abort_flag));
+      ok = __all_sync(0xffffffffu, mbar_wait(&sm.o_full[t], 0, abort_flag));  // one commit, after the last P V
       tc_fence_after();
     }
     // Epilogue: O / l -> bf16.  Each warp stages its 32 rows in this tile's
