@@ -116,8 +116,10 @@ struct __align__(1024) Smem {
   __nv_bfloat16 k[C::kStages][C::kChunks][kBN * 64];
   __nv_bfloat16 v[C::kStages][C::kChunks][kBN * 64];
   uint64_t q_full[2];
-  uint64_t k_full[C::kStages], k_empty[C::kStages];
-  uint64_t v_full[C::kStages], v_empty[C::kStages];
+  uint64_t k_full[C::kStages], v_full[C::kStages];
+  // kv_done[i % kStages] completes when key iteration i has finished with
+  // K(i) and V(i - 1): one commit per iteration frees a K slot and a V slot
+  uint64_t kv_done[C::kStages];
   uint64_t s_full[2], p_full[2][kPChunks], o_full[2];
   uint64_t mma_done;
   uint64_t v_tail;  // paged: V tile holding the sequence end, before its tail is cleared
@@ -200,9 +202,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int s = 0; s < C::kStages; ++s) {
       mbar_init(&sm.k_full[s], 1);
-      mbar_init(&sm.k_empty[s], 1);
+      mbar_init(&sm.kv_done[s], 1);
       mbar_init(&sm.v_full[s], 1);
-      mbar_init(&sm.v_empty[s], 1);
     }
     mbar_init(&sm.mma_done, 1);
     mbar_init(&sm.v_tail, 1);
@@ -306,7 +307,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t tile_bytes = static_cast<uint32_t>(nblk) * 16 * D * 2;
       bool ok = true;
       if (lane == 0) {
-        ok = mbar_wait(&sm.k_empty[s], ph ^ 1, abort_flag);
+        ok = mbar_wait(&sm.kv_done[s], ph ^ 1, abort_flag);  // iteration j - kStages freed K's slot
         if (ok) {
           mbar_arrive_expect_tx(&sm.k_full[s], tile_bytes);
           for (int c = 0; c < C::kChunks; ++c) {
@@ -319,7 +320,11 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
           }
           k_issued = j + 1;
-          ok = mbar_wait(&sm.v_empty[s], ph ^ 1, abort_flag);
+          // V(j) reuses V(j - kStages)'s slot, freed by iteration j - kStages + 1
+          if (j >= C::kStages) {
+            const int it = j - C::kStages + 1;
+            ok = mbar_wait(&sm.kv_done[it % C::kStages], (it / C::kStages) & 1, abort_flag);
+          }
         }
       }
       if (!__shfl_sync(0xffffffffu, ok ? 1 : 0, 0)) break;
@@ -430,14 +435,13 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
         if (!ok) break;
-        umma_commit(&sm.k_empty[s]);
-        if (j >= 1) umma_commit(&sm.v_empty[(j - 1) % C::kStages]);
+        umma_commit(&sm.kv_done[s]);  // K(j) and V(j - 1) are free
       }
       if (ok && n_max > 0) {
         const int jl = n_max - 1;
         for (int t = 0; t < 2 && ok; ++t)
           if (jl < nt[t]) ok = issue_pv(t, jl, t == 0 || jl >= nt[0], true);
-        if (ok) umma_commit(&sm.v_empty[jl % C::kStages]);
+
       }
       // Every MMA issued above is complete once mma_done fires; after an
       // abort this keeps tensor memory allocated until they have finished.
