@@ -60,11 +60,11 @@ WORKLOAD_SETS = {
 #   step / fp8: decode split kernel + LSE combine of one paged_attn_decode call
 #   long, varlen, chunked: the prefill launch
 TRAFFIC_BYTES = {
-    "step": 597.40e6 + 3.16e6 + 4.58e6,   # profiles/launches_llama3_8b_prefill_paged_decode_b64.md
+    "step": 597.39e6 + 3.17e6 + 4.58e6,   # profiles/launches_llama3_8b_prefill_paged_decode_b64.md
     "fp8": 299.00e6 + 2.60e6 + 4.58e6,    # profiles/launches_llama3_8b_prefill_paged_decode_b64_fp8.md
-    "long": 370.43e6 + 101.35e6,          # profiles/launches_long_prefill_16k_long_decode_131k.md
-    "varlen": 250.87e6 + 89.28e6,         # profiles/launches_varlen_prefill_16seq_paged_decode_b64.md
-    "chunked": 337.39e6 + 25.07e6,        # profiles/launches_chunked_prefill_paged_paged_decode_b64.md
+    "long": 375.34e6 + 101.33e6,          # profiles/launches_long_prefill_16k_long_decode_131k.md
+    "varlen": 249.76e6 + 89.21e6,         # profiles/launches_varlen_prefill_16seq_paged_decode_b64.md
+    "chunked": 337.44e6 + 25.50e6,        # profiles/launches_chunked_prefill_paged_paged_decode_b64.md
 }
 
 
