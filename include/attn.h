@@ -22,6 +22,11 @@
  *    contiguous, 16-byte aligned base).  Float outputs are fp32.
  *  - Every call is asynchronous on `stream` (a cudaStream_t; 0 = legacy
  *    default stream) and performs no host<->device synchronisation.
+ *  - Kernels are launched as programmatic dependents of the work before them
+ *    on `stream`: their set-up (barriers, tensor memory, L2 prefetches of
+ *    inputs whose addresses need no memory read) may overlap the previous
+ *    kernel's tail, but every read or write of caller memory happens after
+ *    that kernel has completed, so stream order is unchanged for the caller.
  *  - Return value: ATTN_OK (0) or a negative attn_status_t.  Argument errors
  *    are detected on the host before anything is launched; nothing is written
  *    to the outputs in that case.  There is no fallback path: an unsupported
