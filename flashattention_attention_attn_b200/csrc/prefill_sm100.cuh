@@ -284,47 +284,53 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (warp == kWarpLoad) {
     // ------------------------------ producer ------------------------------
-    // The whole warp runs the loop (paged mode loads block ids in parallel);
-    // lane 0 waits on the barriers and issues the copies.
+    // The whole warp runs the loop; lane 0 waits on the barriers.  Contiguous
+    // tiles take one copy per 64-column chunk (lane 0).  Paged tiles take one
+    // copy per 16-token block and chunk: lane L reads table entry L and issues
+    // the copy of (chunk L / 8, block L % 8), so the 16 copies of a tile leave
+    // in one warp instruction instead of one after another.
     const int nt[2] = {n0, n1};
     int k_issued = pre, v_issued = pre;  // K / V tiles whose loads were issued
     bool tail_issued = false;
+    constexpr int kBlocks = kBN / 16;     // 16-token blocks per tile
+    const int cl = lane / kBlocks, il = lane % kBlocks;  // paged: this lane's (chunk, block)
     for (int j = pre; j < n_max; ++j) {
       const int s = j % C::kStages;
       const uint32_t ph = (j / C::kStages) & 1;
-      int nblk = kBN / 16;   // 16-token blocks loaded into this tile
+      int nblk = kBlocks;    // 16-token blocks loaded into this tile
       int valid = kBN;       // keys of this tile inside the sequence
-      int ids[kBN / 16];
+      int my_id = 0;         // paged: physical block of this lane's copy
       if constexpr (MODE == kPaged) {
         valid = min(kBN, S - j * kBN);
         nblk = (valid + 15) / 16;
         const int mine = (lane < nblk) ? __ldg(p.block_table + static_cast<size_t>(b) * p.max_blocks +
-                                               j * (kBN / 16) + lane)
+                                               j * kBlocks + lane)
                                        : 0;
-#pragma unroll
-        for (int i = 0; i < kBN / 16; ++i) ids[i] = __shfl_sync(0xffffffffu, mine, i);
+        my_id = __shfl_sync(0xffffffffu, mine, il);
       }
+      const bool my_copy = MODE == kPaged && cl < C::kChunks && il < nblk;
       const uint32_t tile_bytes = static_cast<uint32_t>(nblk) * 16 * D * 2;
       bool ok = true;
       if (lane == 0) {
         ok = mbar_wait(&sm.kv_done[s], ph ^ 1, abort_flag);  // iteration j - kStages freed K's slot
         if (ok) {
           mbar_arrive_expect_tx(&sm.k_full[s], tile_bytes);
-          for (int c = 0; c < C::kChunks; ++c) {
-            if constexpr (MODE == kPaged) {
-              for (int i = 0; i < nblk; ++i)
-                tma_load_2d(reinterpret_cast<uint8_t*>(sm.k[s][c]) + i * 16 * 128, &tmK, &sm.k_full[s],
-                            hk * D + c * 64, ids[i] * 16);
-            } else {
+          if constexpr (MODE != kPaged) {
+            for (int c = 0; c < C::kChunks; ++c)
               tma_load_4d(sm.k[s][c], &tmK, &sm.k_full[s], c * 64, hk, koff + j * kBN, bc);
-            }
           }
-          k_issued = j + 1;
-          // V(j) reuses V(j - kStages)'s slot, freed by iteration j - kStages + 1
-          if (j >= C::kStages) {
-            const int it = j - C::kStages + 1;
-            ok = mbar_wait(&sm.kv_done[it % C::kStages], (it / C::kStages) & 1, abort_flag);
-          }
+        }
+      }
+      if (!__shfl_sync(0xffffffffu, ok ? 1 : 0, 0)) break;
+      if (my_copy)
+        tma_load_2d(reinterpret_cast<uint8_t*>(sm.k[s][cl]) + il * 16 * 128, &tmK, &sm.k_full[s],
+                    hk * D + cl * 64, my_id * 16);
+      if (lane == 0) {
+        k_issued = j + 1;
+        // V(j) reuses V(j - kStages)'s slot, freed by iteration j - kStages + 1
+        if (j >= C::kStages) {
+          const int it = j - C::kStages + 1;
+          ok = mbar_wait(&sm.kv_done[it % C::kStages], (it / C::kStages) & 1, abort_flag);
         }
       }
       if (!__shfl_sync(0xffffffffu, ok ? 1 : 0, 0)) break;
@@ -333,14 +339,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         // then the rows past the end (pool slots that may hold anything,
         // even NaN, and blocks not loaded) are cleared so that a zero weight
         // cannot meet a NaN, and only then is the tile handed to the MMA.
-        if (lane == 0) {
-          mbar_arrive_expect_tx(&sm.v_tail, tile_bytes);
-          for (int c = 0; c < C::kChunks; ++c)
-            for (int i = 0; i < nblk; ++i)
-              tma_load_2d(reinterpret_cast<uint8_t*>(sm.v[s][c]) + i * 16 * 128, &tmV, &sm.v_tail,
-                          hk * D + c * 64, ids[i] * 16);
-          tail_issued = true;
-        }
+        if (lane == 0) mbar_arrive_expect_tx(&sm.v_tail, tile_bytes);
+        __syncwarp();
+        if (my_copy)
+          tma_load_2d(reinterpret_cast<uint8_t*>(sm.v[s][cl]) + il * 16 * 128, &tmV, &sm.v_tail,
+                      hk * D + cl * 64, my_id * 16);
+        tail_issued = true;
         ok = __shfl_sync(0xffffffffu, mbar_wait(&sm.v_tail, 0, abort_flag) ? 1 : 0, 0) != 0;
         if (!ok) break;
         for (int i = lane; i < (kBN - valid) * C::kChunks * 8; i += 32) {
@@ -351,17 +355,18 @@ __global__ void __launch_bounds__(kThreads, 1)
         fence_proxy_async_smem();  // the generic writes before the tensor core reads the tile
         __syncwarp();
         if (lane == 0) mbar_arrive(&sm.v_full[s]);
-      } else if (lane == 0) {
-        mbar_arrive_expect_tx(&sm.v_full[s], tile_bytes);
-        for (int c = 0; c < C::kChunks; ++c) {
-          if constexpr (MODE == kPaged) {
-            for (int i = 0; i < nblk; ++i)
-              tma_load_2d(reinterpret_cast<uint8_t*>(sm.v[s][c]) + i * 16 * 128, &tmV, &sm.v_full[s],
-                          hk * D + c * 64, ids[i] * 16);
-          } else {
-            tma_load_4d(sm.v[s][c], &tmV, &sm.v_full[s], c * 64, hk, koff + j * kBN, bc);
+      } else {
+        if (lane == 0) {
+          mbar_arrive_expect_tx(&sm.v_full[s], tile_bytes);
+          if constexpr (MODE != kPaged) {
+            for (int c = 0; c < C::kChunks; ++c)
+              tma_load_4d(sm.v[s][c], &tmV, &sm.v_full[s], c * 64, hk, koff + j * kBN, bc);
           }
         }
+        __syncwarp();
+        if (my_copy)
+          tma_load_2d(reinterpret_cast<uint8_t*>(sm.v[s][cl]) + il * 16 * 128, &tmV, &sm.v_full[s],
+                      hk * D + cl * 64, my_id * 16);
       }
       v_issued = j + 1;
     }
