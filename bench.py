@@ -160,6 +160,8 @@ def parse_args():
     ap.add_argument("--workload", choices=sorted(WORKLOAD_SETS), default="step")
     ap.add_argument("--num-splits", type=int, default=0, help="decode splits (0 = library's choice)")
     ap.add_argument("--e2e-steps", type=int, default=5)
+    ap.add_argument("--streams", type=int, choices=[1, 2], default=2,
+                    help="1: prefill then decode on one stream; 2: the two run concurrently (fork/join per step)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     return ap.parse_args()
 
@@ -423,24 +425,41 @@ def main():
     bt, sl = dinp.block_table.to(dev), dinp.seq_lens.to(dev)
     od = torch.empty(ds.B, ds.Hq, ds.d, device=dev, dtype=torch.bfloat16)
     maxb = dinp.block_table.shape[1]
+    # The prefill and the decode of one step touch disjoint data, so with
+    # --streams 2 they run concurrently: the prefill on the current stream,
+    # the decode on a second stream of the same priority that forks from it
+    # and joins it again every step, so the decode's CTAs fill the SMs the
+    # prefill leaves idle.  All timing events sit on the current stream.  (A
+    # higher priority for the prefill's stream measured slower on the default
+    # and FP8 steps.)
     stream = torch.cuda.current_stream(dev)
+    side = torch.cuda.Stream(dev) if args.streams == 2 else stream
+    fork_ev, join_ev = torch.cuda.Event(), torch.cuda.Event()
 
     flops = pre.flops
     dbytes = workloads.decode_bytes(dinp.seq_lens.tolist(), ds.Hq, ds.Hkv, ds.d, ds.block_size,
                                     kv_elem_bytes=1 if dfp8 else 2)
     splits = args.num_splits
 
-    def decode_call():
+    def decode_call(st):
         if dfp8:
             fa.paged_attn_decode_fp8(qd_, kc, vc, bt, sl, ds.B, ds.Hq, ds.Hkv, ds.d, ds.block_size, maxb, splits,
-                                     dinp.k_scale, dinp.v_scale, od, stream)
+                                     dinp.k_scale, dinp.v_scale, od, st)
         else:
             fa.paged_attn_decode(qd_, kc, vc, bt, sl, ds.B, ds.Hq, ds.Hkv, ds.d, ds.block_size, maxb, splits, od,
-                                 stream)
+                                 st)
 
     def step():
+        if side is stream:
+            pre.call(stream)
+            decode_call(stream)
+            return
+        fork_ev.record(stream)
+        side.wait_event(fork_ev)
         pre.call(stream)
-        decode_call()
+        decode_call(side)
+        join_ev.record(side)
+        stream.wait_event(join_ev)
 
     for _ in range(max(3, args.warmup)):
         step()
@@ -470,13 +489,13 @@ def main():
     total_ms = start.elapsed_time(end)
 
     # Per-part split (reported, not the value): K more steps with events
-    # between the parts.
+    # between the parts, both parts on one stream.
     ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(K)]
     for i in range(K):
         ev[i][0].record(stream)
         pre.call(stream)
         ev[i][1].record(stream)
-        decode_call()
+        decode_call(stream)
         ev[i][2].record(stream)
     torch.cuda.synchronize()
     status = fa.attn_read_device_status(clear=True)
@@ -511,13 +530,14 @@ def main():
             dist.barrier()
         torch.cuda.synchronize()
         e0.record(stream)
-        for _ in range(args.e2e_steps):
-            for h, d_ in zip(h_in, d_in):
-                d_.copy_(h, non_blocking=True)
-            step()
-            h_o.copy_(pre.o, non_blocking=True)
-            h_lse.copy_(pre.lse, non_blocking=True)
-            h_od.copy_(od, non_blocking=True)
+        with torch.cuda.stream(stream):  # the copies go on the step's (joining) stream
+            for _ in range(args.e2e_steps):
+                for h, d_ in zip(h_in, d_in):
+                    d_.copy_(h, non_blocking=True)
+                step()
+                h_o.copy_(pre.o, non_blocking=True)
+                h_lse.copy_(pre.lse, non_blocking=True)
+                h_od.copy_(od, non_blocking=True)
         e1.record(stream)
         torch.cuda.synchronize()
         e2e_ms = e0.elapsed_time(e1) / args.e2e_steps
@@ -561,6 +581,8 @@ def main():
         "config": {"workload": f"{pname} + {dname}", "prefill": pre.config,
                    "decode": {**vars_of(ds), "kv_cache": "fp8 e4m3" if dfp8 else "bf16"},
                    "decode_num_splits": splits or "auto", "parallelism": f"replicas x{world} (no exchange)",
+                   "streams": ("prefill and decode concurrently on two streams (fork/join every step)"
+                               if args.streams == 2 else "prefill then decode on one stream"),
                    "l2": "inputs larger than L2 (decode KV cache %.0f MB per step)" % (dbytes / 1e6)},
         "parts": {"prefill": {"ms": t_pre, "tflops": pre_tflops, "frac": pre_tflops / peaks["bf16_tflops"],
                               "flops": flops},
