@@ -248,9 +248,21 @@ int launch_prefill(const void* q, const void* k, const void* v, void* o, float* 
                     dim3(prefill::kThreads), prefill::smem_bytes<D>(), stream, mq, mk, mv, p);
 }
 
-// Packed sequences: the maps see [total, H, D] as one batch; the grid covers
-// ceil(max_seqlen_q / 256) query blocks of every (sequence, head) and CTAs
-// past a sequence's end exit at once.
+// Packed batches of up to 32 sequences launch one CTA per (head, work item),
+// a work item being one 256-row query block of one sequence.  A sequence of
+// l rows has ceil(l / 256) of them, so at most (total_q + 255 B) / 256 exist
+// (at least 1 here: B, total_q >= 1); CTAs past the last one return at once.
+// Larger batches (0) take the full grid of ceil(max_seqlen_q / 256) blocks
+// for every (sequence, head), where CTAs past a sequence's end exit at once.
+int compact_items(int B, int num_mblocks, int total_q) {
+  if (B > 32) return 0;
+  const long long full = static_cast<long long>(num_mblocks) * B;
+  const long long bound = (static_cast<long long>(total_q) + static_cast<long long>(B) * (2 * prefill::kBM - 1)) /
+                          (2 * prefill::kBM);
+  return static_cast<int>(bound < full ? bound : full);
+}
+
+// Packed sequences: the maps see [total, H, D] as one batch.
 template <int D>
 int launch_prefill_varlen(const void* q, const void* k, const void* v, void* o, float* lse, const int32_t* cu_q,
                           const int32_t* cu_k, int B, int max_q, int total_q, int total_k, int Hq, int Hkv,
@@ -274,7 +286,8 @@ int launch_prefill_varlen(const void* q, const void* k, const void* v, void* o, 
   p.causal = causal ? 1 : 0;
   p.scale_log2 = scale * 1.4426950408889634f;
   p.num_mblocks = (max_q + 2 * prefill::kBM - 1) / (2 * prefill::kBM);
-  const long long grid = static_cast<long long>(p.num_mblocks) * Hq * B;
+  p.items = compact_items(B, p.num_mblocks, total_q);
+  const long long grid = static_cast<long long>(p.items > 0 ? p.items : static_cast<long long>(p.num_mblocks) * B) * Hq;
   if (grid > 0x7fffffffLL) return ATTN_ERR_UNSUPPORTED;
   return launch_pdl(prefill::prefill_fwd_sm100<D, prefill::kVarlen>, dim3(static_cast<unsigned>(grid)),
                     dim3(prefill::kThreads), prefill::smem_bytes<D>(), stream, mq, mk, mv, p);
@@ -305,7 +318,8 @@ int launch_prefill_paged(const void* q, const void* kc, const void* vc, const in
   p.causal = causal ? 1 : 0;
   p.scale_log2 = scale * 1.4426950408889634f;
   p.num_mblocks = (max_q + 2 * prefill::kBM - 1) / (2 * prefill::kBM);
-  const long long grid = static_cast<long long>(p.num_mblocks) * Hq * B;
+  p.items = compact_items(B, p.num_mblocks, total_q);
+  const long long grid = static_cast<long long>(p.items > 0 ? p.items : static_cast<long long>(p.num_mblocks) * B) * Hq;
   if (grid > 0x7fffffffLL) return ATTN_ERR_UNSUPPORTED;
   return launch_pdl(prefill::prefill_fwd_sm100<D, prefill::kPaged>, dim3(static_cast<unsigned>(grid)),
                     dim3(prefill::kThreads), prefill::smem_bytes<D>(), stream, mq, mk, mv, p);

@@ -150,6 +150,7 @@ struct Params {
   int causal;
   float scale_log2;  // scale * log2(e)
   int num_mblocks;   // ceil(T / 256)
+  int items;         // packed, B <= 32: grid = Hq x items (see below); 0: grid = Hq x B x num_mblocks
 };
 
 // Keys visible to the query tile with rows [r0, r0 + 128) (ragged T clipped)
@@ -182,12 +183,12 @@ __global__ void __launch_bounds__(kThreads, 1)
   // Work tile: heaviest (last) query blocks first; adjacent CTAs are adjacent
   // q heads of one (block, batch) so the heads sharing a KV head run together.
   const int per_mb = p.Hq * p.B;
-  const int mb = p.num_mblocks - 1 - static_cast<int>(blockIdx.x) / per_mb;
+  int mb = p.num_mblocks - 1 - static_cast<int>(blockIdx.x) / per_mb;
   const int rem = static_cast<int>(blockIdx.x) % per_mb;
   const int h = rem % p.Hq;
-  const int b = rem / p.Hq;
+  int b = rem / p.Hq;
   const int hk = h / (p.Hq / p.Hkv);
-  const int m0 = mb * 2 * kBM;
+  int m0 = mb * 2 * kBM;
   constexpr bool VARLEN = MODE != kDense;  // packed queries and outputs
 
   // Setup that reads no global memory (barriers, tensor memory, descriptor
@@ -235,6 +236,29 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   int T = p.T, S = p.S, qoff = 0, koff = 0, bc = b;  // bc: batch coordinate of the maps
   if constexpr (VARLEN) {
+    if (p.items > 0) {
+      // Compact grid: CTA -> work item blockIdx / Hq -> (sequence, query
+      // block) in the order of the full grid (top query blocks first,
+      // sequences ascending) but without the blocks past a sequence's end.
+      // Lane i holds sequence i's block count; every warp finds the same item.
+      const int len = (lane < p.B) ? p.cu_q[lane + 1] - p.cu_q[lane] : 0;
+      const int nblocks = (len + 2 * kBM - 1) / (2 * kBM);
+      int left = static_cast<int>(blockIdx.x) / p.Hq;
+      b = -1;
+      for (int k = p.num_mblocks - 1; k >= 0 && b < 0; --k) {
+        uint32_t m = __ballot_sync(0xffffffffu, nblocks > k);
+        const int c = __popc(m);
+        if (left < c) {
+          for (int i = 0; i < left; ++i) m &= m - 1;  // drop the first `left` set bits
+          b = __ffs(m) - 1;
+          mb = k;
+        } else {
+          left -= c;
+        }
+      }
+      if (b < 0) return;  // past the last item (the grid is an upper bound)
+      m0 = mb * 2 * kBM;
+    }
     qoff = p.cu_q[b];
     T = p.cu_q[b + 1] - qoff;
     if constexpr (MODE == kPaged) {

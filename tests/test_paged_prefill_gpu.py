@@ -35,6 +35,19 @@ def test_d64_gqa8():
     check_close(f64(o), O, lse.numpy(), L, what="chunked d64")
 
 
+@pytest.mark.parametrize("B", [32, 33])
+def test_many_sequences_both_grids(B):
+    g = torch.Generator().manual_seed(43 + B)
+    ctx = [int(x) for x in torch.randint(1, 700, (B,), generator=g)]
+    ql = [min(c, int(x)) for c, x in zip(ctx, torch.randint(1, 400, (B,), generator=g))]
+    ctx[-1], ql[-1] = 600, 300
+    spec = _spec(B, Hq=8, Hkv=2, seed=43 + B)
+    inp = inputs.make_chunked(spec, ctx_lens=ctx, q_lens=ql)
+    o, lse = run_chunked(inp, True, spec.scale)
+    O, L = oracle_chunked(inp, True, spec.scale)
+    check_close(f64(o), O, lse.numpy(), L, what=f"chunked B={B}")
+
+
 def test_block_permutation_bit_exact_and_nan_tail():
     ctx, ql = [250, 333, 1000], [90, 333, 257]
     spec = _spec(3, seed=42)

@@ -34,6 +34,23 @@ def test_chunked_queries_longer_keys_and_rows_without_keys():
     check_close(f64(o), O, lse.numpy(), L, what="varlen chunked")
 
 
+@pytest.mark.parametrize("B", [32, 40])
+def test_many_sequences_both_grids(B):
+    # up to 32 sequences: one CTA per (head, 256-row query block that exists);
+    # more: the full grid, whose CTAs past a sequence's end exit at once
+    g = torch.Generator().manual_seed(34 + B)
+    lens = [int(x) for x in torch.randint(0, 600, (B,), generator=g)]
+    lens[0], lens[5], lens[-1] = 0, 256, 257
+    spec = _spec(B, Hq=8, Hkv=2, seed=34 + B)
+    inp = inputs.make_varlen(spec, q_lens=lens)
+    o, lse = run_varlen(inp, True, spec.scale)
+    O, L = oracle_varlen(inp, True, spec.scale)
+    check_close(f64(o), O, lse.numpy(), L, what=f"varlen B={B}")
+    # a max_seqlen_q above the true maximum changes nothing
+    o2, lse2 = run_varlen(inp, True, spec.scale, max_q=inp.max_q + 700)
+    assert torch.equal(o, o2) and torch.equal(lse, lse2)
+
+
 def test_head_dim_64_mha():
     lens = [77, 260, 129]
     spec = _spec(len(lens), Hq=8, Hkv=8, d=64, seed=32)
