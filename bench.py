@@ -60,9 +60,9 @@ WORKLOAD_SETS = {
 #   step / fp8: decode split kernel + LSE combine of one paged_attn_decode call
 #   long, varlen, chunked: the prefill launch
 TRAFFIC_BYTES = {
-    "step": 597.39e6 + 3.17e6 + 4.58e6,   # profiles/launches_llama3_8b_prefill_paged_decode_b64.md
-    "fp8": 299.00e6 + 2.60e6 + 4.58e6,    # profiles/launches_llama3_8b_prefill_paged_decode_b64_fp8.md
-    "long": 375.34e6 + 101.33e6,          # profiles/launches_long_prefill_16k_long_decode_131k.md
+    "step": 597.38e6 + 3.14e6 + 4.58e6,   # profiles/launches_llama3_8b_prefill_paged_decode_b64.md
+    "fp8": 299.00e6 + 2.79e6 + 4.58e6,    # profiles/launches_llama3_8b_prefill_paged_decode_b64_fp8.md
+    "long": 385.56e6 + 101.25e6,          # profiles/launches_long_prefill_16k_long_decode_131k.md
     "varlen": 247.64e6 + 89.08e6,         # profiles/launches_varlen_prefill_16seq_paged_decode_b64.md
     "chunked": 337.31e6 + 24.55e6,        # profiles/launches_chunked_prefill_paged_paged_decode_b64.md
 }
