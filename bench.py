@@ -151,7 +151,7 @@ def load_peaks():
         return dict(FALLBACK_PEAKS), "fallback"
 
 
-def parse_args():
+def parse_args(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=2000)
@@ -163,7 +163,7 @@ def parse_args():
     ap.add_argument("--streams", type=int, choices=[1, 2], default=2,
                     help="1: prefill then decode on one stream; 2: the two run concurrently (fork/join per step)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    return ap.parse_args()
+    return ap.parse_args(argv)
 
 
 # --------------------------------------------------------------------------

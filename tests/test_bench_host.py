@@ -68,3 +68,14 @@ def test_prefill_min_bytes_counts_inputs_once_and_outputs():
     # causal work: sum over rows of (row + 1) visible keys
     assert workloads.visible_pairs(T, S, True) == T * (T + 1) // 2
     assert math.isclose(workloads.prefill_flops(B, Hq, T, S, d, True), 4 * d * Hq * T * (T + 1) / 2)
+
+
+def test_default_run_follows_the_timing_rules():
+    # no flags: one GPU, >= 3 warm-up steps, both ops of a step concurrent,
+    # the library's own split choice, end-to-end leg and CPU baseline on
+    b = _bench()
+    a = b.parse_args([])
+    assert a.gpus == 1 and a.warmup >= 3 and a.steps >= 1 and a.impl == "ours"
+    assert a.streams == 2 and a.num_splits == 0 and a.workload == "step"
+    assert a.e2e_steps > 0 and not a.no_cpu_baseline
+    assert b.parse_args(["--streams", "1"]).streams == 1
