@@ -105,8 +105,6 @@ __device__ __forceinline__ void named_barrier_sync(uint32_t id, uint32_t nthread
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }
 
-// ---------------------------------- TMA ------------------------------------
-// All loads are plain (no .multicast::cluster): every CTA fetches its own tiles.
 // ------------------------ programmatic dependent launch ----------------------
 // A kernel launched with programmatic stream serialization may start while
 // the previous grid on the stream is still running.  It must not touch global
@@ -118,6 +116,8 @@ __device__ __forceinline__ void grid_dependency_wait() { asm volatile("griddepco
 // to complete before it reads anything).
 __device__ __forceinline__ void grid_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
 
+// ---------------------------------- TMA ------------------------------------
+// All loads are plain (no cluster multicast): every CTA fetches its own tiles.
 __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap* map) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
 }
