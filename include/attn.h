@@ -27,6 +27,12 @@
  *    inputs whose addresses need no memory read) may overlap the previous
  *    kernel's tail, but every read or write of caller memory happens after
  *    that kernel has completed, so stream order is unchanged for the caller.
+ *  - Calls on different streams may run at the same time (for example a
+ *    prefill on one stream and a decode on another): each call's temporary
+ *    memory is allocated and freed in the order of its own stream.  The one
+ *    exception is paged_attn_decode_noalloc, whose calls share one scratch
+ *    buffer (see there).  The per-device host state is set up once under a
+ *    lock, so calls may also come from several host threads.
  *  - Return value: ATTN_OK (0) or a negative attn_status_t.  Argument errors
  *    are detected on the host before anything is launched; nothing is written
  *    to the outputs in that case.  There is no fallback path: an unsupported
