@@ -1,7 +1,6 @@
 """Parity of the sm_100a paged decode (paged_attn_decode through the C ABI)
 with the fp64 oracle, split invariance and block-table bit-exactness."""
 
-import numpy as np
 import pytest
 import torch
 
