@@ -91,6 +91,88 @@ def test_paged_decode_host_validation(lib, kw, expect):
     assert _dec(lib, **kw) == expect
 
 
+def _varlen(lib, ptrs=(1 << 20,) * 7, B=2, max_q=64, total_q=100, total_k=100, Hq=8, Hkv=2, d=128, scale=0.088):
+    q, k, v, o, lse, cq, ck = ptrs
+    return lib.attn_fwd_varlen(q, k, v, o, lse, cq, ck, B, max_q, total_q, total_k, Hq, Hkv, d, 1,
+                               ctypes.c_float(scale), None)
+
+
+@pytest.mark.parametrize("kw,expect", [
+    (dict(ptrs=(None,) + (1 << 20,) * 6), INVALID),          # q
+    (dict(ptrs=(1 << 20,) * 5 + (None, 1 << 20)), INVALID),  # cu_seqlens_q
+    (dict(ptrs=(1 << 20, None) + (1 << 20,) * 5), INVALID),  # k with keys present
+    (dict(total_k=-1), INVALID),
+    (dict(Hkv=3), INVALID),
+    (dict(scale=-1.0), INVALID),
+    (dict(d=256), UNSUPPORTED),
+    (dict(ptrs=(1 << 20,) * 5 + (2 + (1 << 20), 1 << 20)), UNSUPPORTED),  # cu_seqlens_q not 4-byte aligned
+    (dict(ptrs=(1 << 20,) * 4 + (1 + (1 << 20),) + (1 << 20,) * 2), UNSUPPORTED),  # lse not 4-byte aligned
+    (dict(B=0), OK),
+    (dict(total_q=0), OK),
+    (dict(max_q=0), OK),
+])
+def test_attn_fwd_varlen_host_validation(lib, kw, expect):
+    assert _varlen(lib, **kw) == expect
+
+
+def _chunked(lib, ptrs=(1 << 20,) * 8, B=2, Hq=8, Hkv=2, d=128, bs=16, maxb=8, max_q=32, total_q=40, scale=0.088):
+    q, kc, vc, bt, sl, cq, o, lse = ptrs
+    return lib.paged_attn_prefill(q, kc, vc, bt, sl, cq, B, Hq, Hkv, d, bs, maxb, max_q, total_q, 1,
+                                  ctypes.c_float(scale), o, lse, None)
+
+
+@pytest.mark.parametrize("kw,expect", [
+    (dict(ptrs=(1 << 20,) * 3 + (None,) + (1 << 20,) * 4), INVALID),  # block_table
+    (dict(ptrs=(1 << 20,) * 6 + (None, 1 << 20)), INVALID),           # o
+    (dict(maxb=0), INVALID),
+    (dict(Hq=9), INVALID),
+    (dict(scale=float("nan")), INVALID),
+    (dict(bs=8), UNSUPPORTED),
+    (dict(d=32), UNSUPPORTED),
+    (dict(ptrs=(1 << 20, 8 + (1 << 20)) + (1 << 20,) * 6), UNSUPPORTED),  # k_cache not 16-byte aligned
+    (dict(B=0), OK),
+    (dict(total_q=0), OK),
+])
+def test_paged_prefill_host_validation(lib, kw, expect):
+    assert _chunked(lib, **kw) == expect
+
+
+def _fp8(lib, ptrs=(1 << 20,) * 6, B=2, Hq=32, Hkv=8, d=128, bs=16, maxb=8, splits=0, ks=0.5, vs=2.0):
+    q, kc, vc, bt, sl, o = ptrs
+    return lib.paged_attn_decode_fp8(q, kc, vc, bt, sl, B, Hq, Hkv, d, bs, maxb, splits, ctypes.c_float(ks),
+                                     ctypes.c_float(vs), o, None)
+
+
+@pytest.mark.parametrize("kw,expect", [
+    (dict(ptrs=(1 << 20,) * 4 + (None, 1 << 20)), INVALID),  # seq_lens
+    (dict(ks=0.0), INVALID),
+    (dict(vs=float("inf")), INVALID),
+    (dict(maxb=-1), INVALID),
+    (dict(d=64), UNSUPPORTED),       # the FP8 path is built for d = 128
+    (dict(bs=32), UNSUPPORTED),
+    (dict(Hq=80, Hkv=8), UNSUPPORTED),  # group of 10 query heads > 8
+    (dict(B=0), OK),
+])
+def test_paged_decode_fp8_host_validation(lib, kw, expect):
+    assert _fp8(lib, **kw) == expect
+
+
+@pytest.mark.parametrize("kw,expect", [
+    (dict(ptrs=(16, 16, None, 16, 16, 16)), INVALID),
+    (dict(Hkv=5), INVALID),
+    (dict(d=80), UNSUPPORTED),
+    (dict(B=0), OK),
+])
+def test_paged_decode_noalloc_host_validation(lib, kw, expect):
+    ptrs = kw.pop("ptrs", (1 << 20,) * 6)
+    args = dict(B=2, Hq=32, Hkv=8, d=128, bs=16, maxb=8, splits=0)
+    args.update(kw)
+    q, kc, vc, bt, sl, o = ptrs
+    rc = lib.paged_attn_decode_noalloc(q, kc, vc, bt, sl, args["B"], args["Hq"], args["Hkv"], args["d"], args["bs"],
+                                       args["maxb"], args["splits"], o, None)
+    assert rc == expect
+
+
 def test_no_cpu_fallback_without_device(lib):
     """Valid arguments without a usable device fail loudly (no silent CPU path)."""
     import torch
@@ -98,4 +180,7 @@ def test_no_cpu_fallback_without_device(lib):
         pytest.skip("a GPU is present")
     assert _fwd(lib) < 0
     assert _dec(lib) < 0
+    assert _varlen(lib) < 0
+    assert _chunked(lib) < 0
+    assert _fp8(lib) < 0
     assert lib.attn_check_support(0) < 0
