@@ -4,13 +4,20 @@ give output shapes without running anything) and with CUDA-graph capture.
 
     import flashattention_attention_attn_b200.torch_ops  # registers the ops
     o, lse = torch.ops.fa_b200.attn_fwd(q, k, v, causal, scale)
+    o, lse = torch.ops.fa_b200.attn_fwd_varlen(q, k, v, cu_seqlens_q, cu_seqlens_k, max_seqlen_q, causal, scale)
+    o, lse = torch.ops.fa_b200.paged_attn_prefill(q, k_cache, v_cache, block_table, seq_lens, cu_seqlens_q,
+                                                  max_seqlen_q, causal, scale)
     o = torch.ops.fa_b200.paged_attn_decode(q, k_cache, v_cache, block_table, seq_lens, num_splits)
+    o = torch.ops.fa_b200.paged_attn_decode_fp8(q, k_cache, v_cache, block_table, seq_lens, num_splits,
+                                                k_scale, v_scale)
 
 The op bodies only allocate the outputs and call the library on the current
 stream; there is no other path.  Shapes follow include/attn.h:
 q [B,T,Hq,d], k/v [B,S,Hkv,d] -> o [B,T,Hq,d], lse [B,Hq,T];
-decode q [B,Hq,d], caches [num_blocks,16,Hkv,d], block_table [B,max_blocks],
-seq_lens [B] -> o [B,Hq,d].
+packed q [total_q,Hq,d], k/v [total_k,Hkv,d], cu_seqlens int32 [B+1]
+-> o [total_q,Hq,d], lse [Hq,total_q];
+decode q [B,Hq,d], caches [num_blocks,16,Hkv,d] (bf16, or e4m3 bytes),
+block_table [B,max_blocks], seq_lens [B] -> o [B,Hq,d].
 """
 
 from __future__ import annotations
@@ -51,4 +58,62 @@ def paged_attn_decode(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Ten
 
 @paged_attn_decode.register_fake
 def _(q, k_cache, v_cache, block_table, seq_lens, num_splits):
+    return torch.empty_like(q)
+
+
+@torch.library.custom_op("fa_b200::attn_fwd_varlen", mutates_args=())
+def attn_fwd_varlen(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, cu_seqlens_q: torch.Tensor,
+                    cu_seqlens_k: torch.Tensor, max_seqlen_q: int, causal: bool,
+                    scale: float) -> tuple[torch.Tensor, torch.Tensor]:
+    total_q, Hq, d = q.shape
+    total_k, Hkv = k.shape[0], k.shape[1]
+    B = cu_seqlens_q.shape[0] - 1
+    o = torch.empty_like(q)
+    lse = torch.empty((Hq, total_q), device=q.device, dtype=torch.float32)
+    _binding.attn_fwd_varlen(q, k, v, o, lse, cu_seqlens_q, cu_seqlens_k, B, max_seqlen_q, total_q, total_k, Hq,
+                             Hkv, d, causal, scale, torch.cuda.current_stream(q.device))
+    return o, lse
+
+
+@attn_fwd_varlen.register_fake
+def _(q, k, v, cu_seqlens_q, cu_seqlens_k, max_seqlen_q, causal, scale):
+    total_q, Hq, _ = q.shape
+    return torch.empty_like(q), q.new_empty((Hq, total_q), dtype=torch.float32)
+
+
+@torch.library.custom_op("fa_b200::paged_attn_prefill", mutates_args=())
+def paged_attn_prefill(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor, block_table: torch.Tensor,
+                       seq_lens: torch.Tensor, cu_seqlens_q: torch.Tensor, max_seqlen_q: int, causal: bool,
+                       scale: float) -> tuple[torch.Tensor, torch.Tensor]:
+    total_q, Hq, d = q.shape
+    Hkv, block_size = k_cache.shape[2], k_cache.shape[1]
+    B = cu_seqlens_q.shape[0] - 1
+    o = torch.empty_like(q)
+    lse = torch.empty((Hq, total_q), device=q.device, dtype=torch.float32)
+    _binding.paged_attn_prefill(q, k_cache, v_cache, block_table, seq_lens, cu_seqlens_q, B, Hq, Hkv, d, block_size,
+                                block_table.shape[1], max_seqlen_q, total_q, causal, scale, o, lse,
+                                torch.cuda.current_stream(q.device))
+    return o, lse
+
+
+@paged_attn_prefill.register_fake
+def _(q, k_cache, v_cache, block_table, seq_lens, cu_seqlens_q, max_seqlen_q, causal, scale):
+    total_q, Hq, _ = q.shape
+    return torch.empty_like(q), q.new_empty((Hq, total_q), dtype=torch.float32)
+
+
+@torch.library.custom_op("fa_b200::paged_attn_decode_fp8", mutates_args=())
+def paged_attn_decode_fp8(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor, block_table: torch.Tensor,
+                          seq_lens: torch.Tensor, num_splits: int, k_scale: float, v_scale: float) -> torch.Tensor:
+    B, Hq, d = q.shape
+    Hkv, block_size = k_cache.shape[2], k_cache.shape[1]
+    o = torch.empty_like(q)
+    _binding.paged_attn_decode_fp8(q, k_cache, v_cache, block_table, seq_lens, B, Hq, Hkv, d, block_size,
+                                   block_table.shape[1], num_splits, k_scale, v_scale, o,
+                                   torch.cuda.current_stream(q.device))
+    return o
+
+
+@paged_attn_decode_fp8.register_fake
+def _(q, k_cache, v_cache, block_table, seq_lens, num_splits, k_scale, v_scale):
     return torch.empty_like(q)

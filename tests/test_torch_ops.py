@@ -22,6 +22,18 @@ def test_fake_shapes_without_running_anything():
         bt = torch.empty(5, 8, dtype=torch.int32)
         od = torch.ops.fa_b200.paged_attn_decode(qd, kc, kc, bt, torch.empty(5, dtype=torch.int32), 0)
         assert od.shape == qd.shape
+        # packed and paged prefill: o like q, lse [Hq, total_q]
+        qp = torch.empty(700, 32, 128, dtype=torch.bfloat16)
+        kp = torch.empty(900, 8, 128, dtype=torch.bfloat16)
+        cu = torch.empty(4, dtype=torch.int32)
+        o, lse = torch.ops.fa_b200.attn_fwd_varlen(qp, kp, kp, cu, cu, 300, True, 0.088)
+        assert o.shape == qp.shape and lse.shape == (32, 700) and lse.dtype == torch.float32
+        o, lse = torch.ops.fa_b200.paged_attn_prefill(qp, kc, kc, torch.empty(3, 8, dtype=torch.int32),
+                                                      torch.empty(3, dtype=torch.int32), cu, 300, True, 0.088)
+        assert o.shape == qp.shape and lse.shape == (32, 700)
+        k8 = torch.empty(40, 16, 8, 128, dtype=torch.uint8)
+        od = torch.ops.fa_b200.paged_attn_decode_fp8(qd, k8, k8, bt, torch.empty(5, dtype=torch.int32), 0, 0.5, 2.0)
+        assert od.shape == qd.shape and od.dtype == torch.bfloat16
 
 
 @pytest.mark.gpu
@@ -48,3 +60,32 @@ def test_ops_match_binding_and_compile_without_graph_break():
     o, lse, od = g(q, k, v, dq, kc, vc, bt, sl)
     torch.cuda.synchronize()
     assert torch.equal(o, o_ref) and torch.equal(lse, lse_ref) and torch.equal(od, od_ref)
+
+
+@pytest.mark.gpu
+def test_packed_chunked_and_fp8_ops_match_the_binding():
+    from tests._parity import run_chunked, run_decode_fp8, run_varlen
+    vs = inputs.VarlenSpec(B=3, Hq=8, Hkv=2, d=128, len_lo=1, len_hi=1, causal=True, seed=62)
+    vin = inputs.make_varlen(vs, q_lens=[5, 130, 300])
+    o_ref, lse_ref = run_varlen(vin, True, vs.scale)
+    o, lse = torch.ops.fa_b200.attn_fwd_varlen(vin.q.cuda(), vin.k.cuda(), vin.v.cuda(), vin.cu_q.cuda(),
+                                               vin.cu_k.cuda(), vin.max_q, True, vs.scale)
+    assert torch.equal(o.cpu(), o_ref) and torch.equal(lse.cpu(), lse_ref)
+
+    cs = inputs.ChunkedSpec(B=2, Hq=8, Hkv=2, d=128, block_size=16, max_blocks=32, ctx_lo=1, ctx_hi=1, q_lo=1, q_hi=1,
+                            seed=63)
+    cin = inputs.make_chunked(cs, ctx_lens=[300, 77], q_lens=[100, 77])
+    o_ref, lse_ref = run_chunked(cin, True, cs.scale)
+    c = cin.cache
+    o, lse = torch.ops.fa_b200.paged_attn_prefill(cin.q.cuda(), c.k_cache.cuda(), c.v_cache.cuda(),
+                                                  c.block_table.cuda(), c.seq_lens.cuda(), cin.cu_q.cuda(),
+                                                  cin.max_q, True, cs.scale)
+    assert torch.equal(o.cpu(), o_ref) and torch.equal(lse.cpu(), lse_ref)
+
+    ds = inputs.DecodeSpec(B=3, Hq=32, Hkv=8, d=128, block_size=16, max_blocks=16, ctx_lo=10, ctx_hi=250, seed=64)
+    din = inputs.make_paged_fp8(ds)
+    od_ref = run_decode_fp8(din, num_splits=0)
+    od = torch.ops.fa_b200.paged_attn_decode_fp8(din.q.cuda(), din.k_cache.cuda(), din.v_cache.cuda(),
+                                                 din.block_table.cuda(), din.seq_lens.cuda(), 0, din.k_scale,
+                                                 din.v_scale)
+    assert torch.equal(od.cpu(), od_ref)
