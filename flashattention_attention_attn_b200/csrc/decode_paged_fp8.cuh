@@ -4,9 +4,10 @@
 //
 // Same work decomposition as paged_decode_split (decode_paged.cuh): one CTA
 // per (split, group of kKH kv heads, sequence); a producer warp reads the
-// block table and issues one TMA per head per tensor per 16-token block
-// (a head row of e4m3 is exactly one 128-byte swizzle row); one consumer
-// warp per kv head serves all G = Hq/Hkv query heads of that kv head.
+// block table and issues one TMA per tensor per 16-token block, covering the
+// group's kKH heads (a head row of e4m3 is exactly one 128-byte swizzle
+// row); one consumer warp per kv head serves all G = Hq/Hkv query heads of
+// that kv head.
 //
 // Scores: S^T[16 tokens x 8 heads] = K q^T with f16 mma.sync.  ldmatrix on
 // the e4m3 tile gives each lane 4 consecutive bytes (head-dim columns
