@@ -184,3 +184,21 @@ def test_no_cpu_fallback_without_device(lib):
     assert _chunked(lib) < 0
     assert _fp8(lib) < 0
     assert lib.attn_check_support(0) < 0
+
+
+def test_plain_c_client_compiles_links_and_runs(lib, tmp_path):
+    """include/attn.h compiles as C99 and the library answers a C program."""
+    import shutil
+    import subprocess
+    from flashattention_attention_attn_b200 import _binding
+    cc = shutil.which("gcc") or shutil.which("cc")
+    if cc is None:
+        pytest.skip("no C compiler")
+    src = os.path.join(ROOT, "tests", "c_client", "abi_client.c")
+    exe = str(tmp_path / "abi_client")
+    libdir = os.path.dirname(_binding.library_path)
+    subprocess.run([cc, "-std=c99", "-Wall", "-Wextra", "-Werror", "-I", os.path.join(ROOT, "include"), src,
+                    "-o", exe, "-L", libdir, "-lattn_b200", "-Wl,-rpath," + libdir], check=True)
+    r = subprocess.run([exe], capture_output=True, text=True, timeout=120)
+    assert r.returncode == 0, r.stdout + r.stderr
+    assert "attn_check_support(0)" in r.stdout
