@@ -34,14 +34,8 @@ namespace decode {
 // Stages in flight and resident CTAs per SM.  5 x 16 KB per CTA measured
 // best: 82% vs 78% of the HBM copy peak with 6 on long_decode_131k, equal on
 // paged_decode_b64; 4 stages with 3 CTAs or 3 with 4 gained nothing.
-#ifndef ATTN_FP8_STAGES
-#define ATTN_FP8_STAGES 5
-#endif
-#ifndef ATTN_FP8_CTAS_PER_SM
-#define ATTN_FP8_CTAS_PER_SM 2
-#endif
-constexpr int kFp8Stages = ATTN_FP8_STAGES;        // 16 KB per stage (K + V of 4 heads)
-constexpr int kFp8CtasPerSm = ATTN_FP8_CTAS_PER_SM;  // resident CTAs per SM
+constexpr int kFp8Stages = 5;     // 16 KB per stage (K + V of 4 heads)
+constexpr int kFp8CtasPerSm = 2;  // resident CTAs per SM
 constexpr int kFp8D = 128;      // head dim served by the FP8 path
 constexpr uint32_t kFp8HeadBytes = kBlock * kFp8D;  // one head of one block: 16 rows x 128 B
 

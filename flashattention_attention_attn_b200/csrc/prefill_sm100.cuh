@@ -34,8 +34,6 @@
 // sum always share the same reference, so the final O / l is unchanged.
 #pragma once
 
-#include <type_traits>
-
 #include "sm100_ptx.cuh"
 
 namespace attn {
@@ -48,58 +46,6 @@ constexpr int kWarpLoad = 8;
 constexpr int kWarpMma = 9;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
 constexpr uint32_t kTmemCols = 512;
-
-// Of every 4 pairs of scores in a row chunk, this many take their 2^x from
-// the polynomial below (FMA pipe) instead of ex2 (MUFU), so that both units
-// share the exponentials of tiles that need no mask.
-#ifndef ATTN_PREFILL_POLY_PAIRS
-#define ATTN_PREFILL_POLY_PAIRS 0
-#endif
-constexpr int kPolyPairsOf4 = ATTN_PREFILL_POLY_PAIRS;
-
-// P is handed to the MMA warp in this many column chunks per tile, so that
-// P V of the first chunks runs while the softmax finishes the later ones.
-#ifndef ATTN_PREFILL_P_CHUNKS
-#define ATTN_PREFILL_P_CHUNKS 1
-#endif
-constexpr int kPChunks = ATTN_PREFILL_P_CHUNKS;
-static_assert(kPChunks == 1 || kPChunks == 2 || kPChunks == 4, "P chunks must divide 4");
-
-// 2^x on the FMA pipe: x = j + f with j = round(x) (added into the exponent
-// bits) and f in [-1/2, 1/2]; 2^f by a degree-3 polynomial, minimax in
-// relative error (Remez exchange; coefficients from csrc/gen_exp2_poly.py),
-// max relative error 1.5e-4 in float32 -- far below the bf16 rounding of P.
-// Valid for x in [-126, 127]; smaller x is clamped (result ~2^-126), so it is
-// only used where no score is masked.
-__device__ __forceinline__ float exp2_poly(float x) {
-  constexpr float kC0 = 9.999280572e-01f, kC1 = 6.932609677e-01f;
-  constexpr float kC2 = 2.426111251e-01f, kC3 = 5.517166853e-02f;
-  constexpr float kRound = 12582912.0f;  // 1.5 * 2^23: adding it rounds to an integer
-  x = fmaxf(x, -126.0f);
-  const float t = __fadd_rn(x, kRound);
-  const float j = __fadd_rn(t, -kRound);
-  const float f = __fadd_rn(x, -j);
-  float p = fmaf(kC3, f, kC2);
-  p = fmaf(p, f, kC1);
-  p = fmaf(p, f, kC0);
-  return __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
-}
-
-// The same for a pair, with packed fp32 arithmetic.
-__device__ __forceinline__ float2 exp2_poly2(float2 x) {
-  const float2 kRound = make_float2(12582912.0f, 12582912.0f);
-  const float2 kNegRound = make_float2(-12582912.0f, -12582912.0f);
-  x = make_float2(fmaxf(x.x, -126.0f), fmaxf(x.y, -126.0f));
-  const float2 t = __fadd2_rn(x, kRound);
-  const float2 j = __fadd2_rn(t, kNegRound);
-  const float2 f = __fadd2_rn(x, make_float2(-j.x, -j.y));
-  float2 p = __ffma2_rn(make_float2(5.517166853e-02f, 5.517166853e-02f), f,
-                        make_float2(2.426111251e-01f, 2.426111251e-01f));
-  p = __ffma2_rn(p, f, make_float2(6.932609677e-01f, 6.932609677e-01f));
-  p = __ffma2_rn(p, f, make_float2(9.999280572e-01f, 9.999280572e-01f));
-  return make_float2(__int_as_float(__float_as_int(p.x) + (__float_as_int(t.x) << 23)),
-                     __int_as_float(__float_as_int(p.y) + (__float_as_int(t.y) << 23)));
-}
 
 template <int D>
 struct Config {
@@ -120,7 +66,7 @@ struct __align__(1024) Smem {
   // kv_done[i % kStages] completes when key iteration i has finished with
   // K(i) and V(i - 1): one commit per iteration frees a K slot and a V slot
   uint64_t kv_done[C::kStages];
-  uint64_t s_full[2], p_full[2][kPChunks], o_full[2];
+  uint64_t s_full[2], p_full[2], o_full[2];
   uint64_t mma_done;
   uint64_t v_tail;  // paged: V tile holding the sequence end, before its tail is cleared
   uint32_t tmem_base;
@@ -198,7 +144,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int t = 0; t < 2; ++t) {
       mbar_init(&sm.q_full[t], 1);
       mbar_init(&sm.s_full[t], 1);
-      for (int c = 0; c < kPChunks; ++c) mbar_init(&sm.p_full[t][c], 4);  // one arrive per softmax warp
+      mbar_init(&sm.p_full[t], 4);  // one arrive per softmax warp
       mbar_init(&sm.o_full[t], 1);
     }
     for (int s = 0; s < C::kStages; ++s) {
@@ -424,19 +370,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t tS = tmem + t * kBN;
         const uint32_t tO = tmem + 2 * kBN + t * D;
         const uint32_t vbase = smem_u32(sm.v[s][0]);
-        constexpr int kSteps = kBN / 16 / kPChunks;  // K=16 MMAs per P chunk
+        if (!mbar_wait(&sm.p_full[t], jj & 1, abort_flag)) return false;
+        tc_fence_after();
 #pragma unroll
-        for (int c = 0; c < kPChunks; ++c) {
-          if (!mbar_wait(&sm.p_full[t][c], jj & 1, abort_flag)) return false;
-          tc_fence_after();
-#pragma unroll
-          for (int k2 = 0; k2 < kSteps; ++k2) {
-            const int kk = c * kSteps + k2;
-            // 16 keys per step: 16 rows x 128 B further into each V chunk;
-            // LBO = distance between 64-wide d chunks, SBO = 8 rows x 128 B.
-            const uint64_t bdesc = make_sdesc_sw128(vbase + kk * 16 * 128, C::kChunkBytes, 1024);
-            umma_ts(tO, tS + kk * 8, bdesc, idesc_pv, (jj > 0 || kk > 0) ? 1u : 0u);
-          }
+        for (int kk = 0; kk < kBN / 16; ++kk) {
+          // 16 keys per step: 16 rows x 128 B further into each V chunk;
+          // LBO = distance between 64-wide d chunks, SBO = 8 rows x 128 B.
+          const uint64_t bdesc = make_sdesc_sw128(vbase + kk * 16 * 128, C::kChunkBytes, 1024);
+          umma_ts(tO, tS + kk * 8, bdesc, idesc_pv, (jj > 0 || kk > 0) ? 1u : 0u);
         }
         if (last) umma_commit(&sm.o_full[t]);
         return true;
@@ -547,41 +488,22 @@ __global__ void __launch_bounds__(kThreads, 1)
       const float2 nm2 = make_float2(-mref, -mref);
       float2 sum4[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
                         make_float2(0.f, 0.f)};
-      auto exp_store = [&](auto poly_pairs) {
-        constexpr int kPoly = decltype(poly_pairs)::value;  // pairs of every 4 on the FMA pipe
 #pragma unroll
-        for (int c = 0; c < kBN / 32; ++c) {
-          uint32_t pk[16];
+      for (int c = 0; c < kBN / 32; ++c) {
+        uint32_t pk[16];
 #pragma unroll
-          for (int i = 0; i < 16; ++i) {
-            const float2 x = __ffma2_rn(make_float2(s[c * 32 + 2 * i], s[c * 32 + 2 * i + 1]), c2, nm2);
-            float2 pp;
-            if constexpr (kPoly > 0) {
-              if ((i & 3) < kPoly) pp = exp2_poly2(x);
-              else pp = make_float2(ex2_approx(x.x), ex2_approx(x.y));
-            } else {
-              pp = make_float2(ex2_approx(x.x), ex2_approx(x.y));
-            }
-            sum4[i & 3] = __fadd2_rn(sum4[i & 3], pp);
-            pk[i] = pack_bf16x2(pp.x, pp.y);
-          }
-          tmem_st_x16(tS + c * 16, pk);  // P overwrites the first 64 columns of S
-          if ((c + 1) % (4 / kPChunks) == 0) {
-            tmem_st_wait();
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&sm.p_full[t][(c + 1) / (4 / kPChunks) - 1]);
-          }
+        for (int i = 0; i < 16; ++i) {
+          const float2 x = __ffma2_rn(make_float2(s[c * 32 + 2 * i], s[c * 32 + 2 * i + 1]), c2, nm2);
+          const float2 pp = make_float2(ex2_approx(x.x), ex2_approx(x.y));
+          sum4[i & 3] = __fadd2_rn(sum4[i & 3], pp);
+          pk[i] = pack_bf16x2(pp.x, pp.y);
         }
-      };
-      // The polynomial clamps its input, so it is only used where no score
-      // of the warp's rows is masked; the choice is warp-uniform because the
-      // tcgen05.st inside is a warp-wide (.sync.aligned) instruction.
-      if (kPolyPairsOf4 > 0 && __all_sync(0xffffffffu, lim >= kBN)) {
-        exp_store(std::integral_constant<int, kPolyPairsOf4>{});
-      } else {
-        exp_store(std::integral_constant<int, 0>{});
+        tmem_st_x16(tS + c * 16, pk);  // P overwrites the first 64 columns of S
       }
+      tmem_st_wait();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&sm.p_full[t]);
       const float2 s01 = __fadd2_rn(sum4[0], sum4[1]);
       const float2 s23 = __fadd2_rn(sum4[2], sum4[3]);
       const float2 sall = __fadd2_rn(s01, s23);
