@@ -753,13 +753,19 @@ int launch_decode_noalloc(const void* q, const void* kc, const void* vc, const i
                           const int32_t* lens, int B, int Hq, int Hkv, int max_blocks, int num_splits, void* o,
                           cudaStream_t stream, int sms, void* scratch) {
   const int groups = (Hkv + decode::kKH - 1) / decode::kKH;
-  if (num_splits <= 0) num_splits = auto_splits(B, groups, max_blocks, sms);
+  const size_t row_bytes = static_cast<size_t>(B) * Hq * (D + 1) * sizeof(float);  // partials of one split
+  if (num_splits <= 0) {
+    // the automatic choice, lowered to what the scratch holds (1 split needs none)
+    num_splits = auto_splits(B, groups, max_blocks, sms);
+    const size_t fit = ATTN_NOALLOC_SCRATCH_BYTES / row_bytes;
+    if (static_cast<size_t>(num_splits) > fit) num_splits = fit >= 2 ? static_cast<int>(fit) : 1;
+  }
   if (num_splits > max_blocks) num_splits = max_blocks;
   const int chunk = (max_blocks + num_splits - 1) / num_splits;
   num_splits = (max_blocks + chunk - 1) / chunk;
   if (num_splits > 65535 || groups > 65535 || B > 65535) return ATTN_ERR_UNSUPPORTED;
   const size_t rows = static_cast<size_t>(num_splits) * B * Hq;
-  if (num_splits > 1 && rows * (D + 1) * sizeof(float) > ATTN_NOALLOC_SCRATCH_BYTES) return ATTN_ERR_UNSUPPORTED;
+  if (num_splits > 1 && num_splits * row_bytes > ATTN_NOALLOC_SCRATCH_BYTES) return ATTN_ERR_UNSUPPORTED;
   CUtensorMap mk, mv;
   if (make_map_decode_bf16(&mk, kc, Hkv, D) || make_map_decode_bf16(&mv, vc, Hkv, D)) return ATTN_ERR_CUDA;
 

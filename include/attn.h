@@ -255,11 +255,12 @@ int paged_attn_decode_fp8(const void* q, const void* k_cache, const void* v_cach
  * library until the process exits).  It calls no cudaMalloc, cudaFree or
  * other allocating routine.
  *
- *   Limit: num_splits * B * Hq * (d + 1) * 4 bytes of partials (with the
- *   split count after num_splits <= 0 is resolved and clamped) must not
- *   exceed ATTN_NOALLOC_SCRATCH_BYTES; a larger request returns
- *   ATTN_ERR_UNSUPPORTED before anything is launched.  With one split no
- *   scratch is used.
+ *   Limit: num_splits * B * Hq * (d + 1) * 4 bytes of partials must not
+ *   exceed ATTN_NOALLOC_SCRATCH_BYTES.  With num_splits <= 0 the automatic
+ *   split count is lowered until its partials fit (down to one split, which
+ *   uses no scratch), so an automatic call never fails on this limit; an
+ *   explicit num_splits whose partials do not fit returns
+ *   ATTN_ERR_UNSUPPORTED before anything is launched.
  *   First call on a device: it looks up the scratch array's device address
  *   (cudaGetSymbolAddress, with that device current) and sets the kernels'
  *   shared-memory limits; make that first call before any stream capture.

@@ -18,23 +18,43 @@ def _bench():
     return mod
 
 
-def test_traffic_table_covers_every_workload_set():
+def test_traffic_entries_name_known_workloads_and_kernels():
     b = _bench()
-    assert set(b.TRAFFIC_BYTES) == set(b.WORKLOAD_SETS)
-    for name, v in b.TRAFFIC_BYTES.items():
-        assert v > 0, name
+    for name, t in b.TRAFFIC.items():
+        assert name in b.WORKLOAD_SETS, name
+        assert set(t) <= {"prefill", "decode", "csrc"} and "csrc" in t, name
+        for part in ("prefill", "decode"):
+            if part in t:
+                assert t[part] > 0, (name, part)
 
 
-def test_measured_traffic_is_at_least_the_algorithmic_decode_bytes():
+def test_traffic_applies_only_to_the_kernels_it_was_captured_on():
+    b = _bench()
+    h = b.csrc_hash()
+    assert len(h) == 16 and h == b.csrc_hash()  # stable for the same sources
+    b.TRAFFIC["long"] = {"prefill": 4.9e8, "decode": 5.4e8, "csrc": h}
+    assert b.traffic_of("long", "prefill")[0] == 4.9e8
+    b.TRAFFIC["long"]["csrc"] = "0" * 16  # captured on other kernels
+    val, note = b.traffic_of("long", "prefill")
+    assert val is None and "changed" in note
+    assert b.traffic_of("no-such-set", "decode")[0] is None
+
+
+def test_measured_decode_traffic_is_at_least_the_algorithmic_bytes():
     # a DRAM count below the bytes the method must read would mean a kernel
     # that skipped work (or a stale table)
     b = _bench()
     from flashattention_attention_attn_b200 import inputs, workloads
-    ds = inputs.WORKLOADS["paged_decode_b64"]
-    d = inputs.make_paged(ds)
-    algo = workloads.decode_bytes(d.seq_lens.tolist(), ds.Hq, ds.Hkv, ds.d, ds.block_size)
-    assert b.TRAFFIC_BYTES["step"] >= algo
-    assert b.TRAFFIC_BYTES["step"] < 1.05 * algo  # K/V read once, partials small
+    for name, (pname, dname) in b.WORKLOAD_SETS.items():
+        t = b.TRAFFIC.get(name)
+        if not t or "decode" not in t:
+            continue
+        base, fp8 = b.decode_workload(dname)
+        ds = inputs.WORKLOADS[base]
+        d = inputs.make_paged(ds)
+        algo = workloads.decode_bytes(d.seq_lens.tolist(), ds.Hq, ds.Hkv, ds.d, ds.block_size,
+                                      kv_elem_bytes=1 if fp8 else 2)
+        assert algo <= t["decode"] < 1.05 * algo, name  # K/V read once, partials small
 
 
 def test_clock_summary_uses_samples_inside_the_window():
@@ -71,11 +91,13 @@ def test_prefill_min_bytes_counts_inputs_once_and_outputs():
 
 
 def test_default_run_follows_the_timing_rules():
-    # no flags: one GPU, >= 3 warm-up steps, both ops of a step concurrent,
-    # the library's own split choice, end-to-end leg and CPU baseline on
+    # no flags: one GPU, >= 3 warm-up steps, the long-context pair (16k-token
+    # prefill, 131k-token decode), both ops of a step concurrent, the
+    # library's own split choice, end-to-end leg and CPU baseline on
     b = _bench()
     a = b.parse_args([])
     assert a.gpus == 1 and a.warmup >= 3 and a.steps >= 1 and a.impl == "ours"
-    assert a.streams == 2 and a.num_splits == 0 and a.workload == "step"
+    assert b.WORKLOAD_SETS[a.workload] == ("long_prefill_16k", "long_decode_131k")
+    assert a.streams == 2 and a.num_splits == 0
     assert a.e2e_steps > 0 and not a.no_cpu_baseline
     assert b.parse_args(["--streams", "1"]).streams == 1

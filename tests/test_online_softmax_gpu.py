@@ -1,0 +1,202 @@
+"""GPU parity of the online-softmax update itself: inputs whose running row
+maximum jumps from one key tile to the next, so that the prefill kernel must
+move its reference maximum and rescale the partial output O and the row sum
+held on chip ("werkt het de statistieken van de softmax bij ... accumuleert de
+bijbehorende uitvoer in het on-chip geheugen", page "Snelle attention-kernels
+en operatorfusie versnellen AI-modellen", section "FlashAttention-type aandacht
+en gepagineerde aandacht"), and calls with a scale other than 1/sqrt(d).
+
+The prefill kernel keeps a reference maximum per row and only moves it (and
+rescales O in tensor memory) when a new 128-key tile raises the row maximum
+by more than 8 in log2 units; with N(0, 1) inputs at scale 1/sqrt(d) that
+never happens.  Each input here is built so that it does, and before the GPU
+call the test replays that rule on the CPU from the exact scores (fp64) to
+check that the rescale is reached: for some rows, and for warps (32
+consecutive rows) in which some rows rescale and others keep their reference
+(the warp then takes the tensor-memory round trip with a factor of 1 for the
+latter).  Every result is compared element by element with the fp64 oracle.
+"""
+
+import math
+
+import numpy as np
+import pytest
+import torch
+
+from flashattention_attention_attn_b200 import inputs
+from tests._parity import (check_close, f64, oracle_chunked, oracle_prefill, oracle_varlen, run_chunked, run_prefill,
+                           run_varlen)
+
+pytestmark = pytest.mark.gpu
+
+TILE = 128        # keys per K/V tile of the prefill kernel
+WARP_ROWS = 32    # rows of one softmax warp (query tiles start at multiples of 128)
+THRESHOLD = 8.0   # log2 units the row max must rise by before the kernel rescales
+MARGIN = 0.5      # keep clear of the threshold, so fp32 rounding cannot flip a decision
+LOG2E = 1.0 / math.log(2.0)
+
+
+def rescale_events(q, k, scale, causal):
+    """Replay the kernel's reference-max rule for one head.
+
+    q [T, d], k [S, d] (fp64 values of the bf16 inputs).  Returns
+    (rows_rescaled, mixed_warps): the number of (row, tile) steps where the
+    reference moves by more than THRESHOLD + MARGIN while it was already
+    finite, and the number of (warp, tile) steps where at least one row of a
+    warp does so and at least one other row's maximum stays below
+    THRESHOLD - MARGIN above its reference.
+    """
+    T, S = q.shape[0], k.shape[0]
+    s = (q @ k.T) * (scale * LOG2E)                       # scores, log2 domain
+    vis = np.array([min(S, i + (S - T) + 1) if causal else S for i in range(T)])
+    s = np.where(np.arange(S)[None, :] < vis[:, None], s, -np.inf)
+    m_used = np.full(T, -np.inf)
+    rows, mixed = 0, 0
+    for j in range(0, (S + TILE - 1) // TILE):
+        mx = s[:, j * TILE:(j + 1) * TILE].max(axis=1)
+        with np.errstate(invalid="ignore"):
+            jump = np.maximum(m_used, mx) - m_used           # nan while both are -inf
+        move = np.nan_to_num(jump, nan=0.0) > THRESHOLD
+        resc = move & np.isfinite(m_used) & (jump > THRESHOLD + MARGIN)
+        keep = np.isfinite(m_used) & (np.nan_to_num(jump, nan=0.0) < THRESHOLD - MARGIN)
+        rows += int(resc.sum())
+        for w0 in range(0, T, WARP_ROWS):
+            if resc[w0:w0 + WARP_ROWS].any() and keep[w0:w0 + WARP_ROWS].any():
+                mixed += 1
+        m_used = np.where(move, np.maximum(m_used, mx), m_used)
+    return rows, mixed
+
+
+def tile_gain(n_tiles, step=3.0):
+    """Factor of key tile t: 1, 1 + step, 1 + 2 step, ... (the row max of
+    N(0, 1) scores rises by more than 8 log2 units from tile to tile)."""
+    return [1.0 + step * t for t in range(n_tiles)]
+
+
+def rising_keys(k, gains):
+    """k [..., S, H, d] with key s multiplied by gains[s // TILE] (bf16 again)."""
+    S = k.shape[-3]
+    g = torch.tensor([gains[s // TILE] for s in range(S)], dtype=torch.float32)
+    shape = [1] * k.dim()
+    shape[-3] = S
+    return (k.float() * g.view(shape)).to(torch.bfloat16)
+
+
+def quiet_odd_rows(q, factor=0.05):
+    """q [..., T, H, d] with every odd query row multiplied by `factor`: those
+    rows' scores stay small, so inside every warp some rows rescale and some
+    do not."""
+    T = q.shape[-3]
+    g = torch.tensor([factor if i % 2 else 1.0 for i in range(T)], dtype=torch.float32)
+    shape = [1] * q.dim()
+    shape[-3] = T
+    return (q.float() * g.view(shape)).to(torch.bfloat16)
+
+
+def _dense(q, k, v, causal, scale, need_rows=1, need_mixed=0):
+    for h in range(q.shape[2]):
+        hk = h // (q.shape[2] // k.shape[2])
+        rows, mixed = rescale_events(f64(q[0, :, h]), f64(k[0, :, hk]), scale, causal)
+        need_rows -= rows
+        need_mixed -= mixed
+    assert need_rows <= 0 and need_mixed <= 0, "inputs do not reach the rescale path"
+    o, lse = run_prefill(q, k, v, causal, scale)
+    O, L = oracle_prefill(q, k, v, causal, scale)
+    check_close(f64(o), O, lse.numpy(), L, what=f"causal={causal} scale={scale}")
+
+
+@pytest.mark.parametrize("causal", [True, False])
+def test_rising_row_max_rescales_output(causal):
+    spec = inputs.PrefillSpec(B=1, Hq=8, Hkv=2, T=700, S=700, d=128, causal=causal, seed=80)
+    q, k, v = inputs.make_prefill(spec)
+    k = rising_keys(k, tile_gain(6))
+    _dense(q, k, v, causal, spec.scale, need_rows=1000)
+
+
+def test_mixed_rows_in_one_warp():
+    spec = inputs.PrefillSpec(B=1, Hq=4, Hkv=1, T=600, S=600, d=128, causal=True, seed=81)
+    q, k, v = inputs.make_prefill(spec)
+    q = quiet_odd_rows(q)
+    k = rising_keys(k, tile_gain(5))
+    _dense(q, k, v, True, spec.scale, need_rows=500, need_mixed=20)
+
+
+def test_mixed_rows_head_dim_64():
+    spec = inputs.PrefillSpec(B=2, Hq=4, Hkv=2, T=520, S=520, d=64, causal=True, seed=82)
+    q, k, v = inputs.make_prefill(spec)
+    q = quiet_odd_rows(q)
+    k = rising_keys(k, tile_gain(5, step=4.0))
+    _dense(q, k, v, True, spec.scale, need_rows=200, need_mixed=10)
+
+
+def test_large_scores_scale_one():
+    # |scores| up to ~100 (natural units): the row max of later tiles often
+    # exceeds the reference by more than 8 log2 units without any shaping
+    spec = inputs.PrefillSpec(B=1, Hq=8, Hkv=2, T=640, S=640, d=128, causal=True, seed=83)
+    q, k, v = inputs.make_prefill(spec)
+    q = (q.float() * 2.0).to(torch.bfloat16)
+    assert np.abs(f64(q[0, :, 0]) @ f64(k[0, :, 0]).T).max() > 80.0
+    _dense(q, k, v, True, 1.0, need_rows=50)
+
+
+@pytest.mark.parametrize("scale", [0.05, 0.3, 1.0])
+def test_scale_argument(scale):
+    # the kernel multiplies by the caller's scale (no hidden 1/sqrt(d))
+    spec = inputs.PrefillSpec(B=2, Hq=8, Hkv=2, T=333, S=333, d=128, causal=True, seed=84)
+    q, k, v = inputs.make_prefill(spec)
+    o, lse = run_prefill(q, k, v, True, scale)
+    O, L = oracle_prefill(q, k, v, True, scale)
+    check_close(f64(o), O, lse.numpy(), L, what=f"scale={scale}")
+    O2, L2 = oracle_prefill(q, k, v, True, spec.scale)
+    assert np.abs(L2 - L)[np.isfinite(L)].max() > 1e-2  # another scale gives another result
+
+
+@pytest.mark.parametrize("scale", [0.05, 1.0])
+def test_scale_argument_head_dim_64_noncausal(scale):
+    spec = inputs.PrefillSpec(B=1, Hq=4, Hkv=4, T=200, S=450, d=64, causal=False, seed=85)
+    q, k, v = inputs.make_prefill(spec)
+    o, lse = run_prefill(q, k, v, False, scale)
+    O, L = oracle_prefill(q, k, v, False, scale)
+    check_close(f64(o), O, lse.numpy(), L, what=f"d64 scale={scale}")
+
+
+def test_varlen_rising_row_max_and_scale():
+    lens = [700, 129, 0, 390, 520]
+    spec = inputs.VarlenSpec(B=len(lens), Hq=8, Hkv=2, d=128, len_lo=1, len_hi=1, causal=True, seed=86)
+    inp = inputs.make_varlen(spec, q_lens=lens)
+    cu = inp.cu_q.tolist()
+    kk = inp.k.clone()
+    for b in range(len(lens)):  # tiles start at each sequence's first key
+        if lens[b]:
+            kk[cu[b]:cu[b + 1]] = rising_keys(inp.k[cu[b]:cu[b + 1]], tile_gain(6))
+    q = quiet_odd_rows(inp.q)
+    inp = inputs.VarlenInputs(q=q, k=kk, v=inp.v, cu_q=inp.cu_q, cu_k=inp.cu_k)
+    rows, mixed = rescale_events(f64(q[cu[0]:cu[1], 0]), f64(kk[cu[0]:cu[1], 0]), 0.3, True)
+    assert rows > 100 and mixed > 5
+    o, lse = run_varlen(inp, True, 0.3)
+    O, L = oracle_varlen(inp, True, 0.3)
+    check_close(f64(o), O, lse.numpy(), L, what="varlen rising")
+
+
+def test_chunked_rising_row_max_and_scale():
+    ctx, ql = [900, 300, 517], [600, 300, 200]
+    spec = inputs.ChunkedSpec(B=3, Hq=8, Hkv=2, d=128, block_size=16, max_blocks=64, ctx_lo=1, ctx_hi=1, q_lo=1,
+                              q_hi=1, seed=87)
+    inp = inputs.make_chunked(spec, ctx_lens=ctx, q_lens=ql)
+    c = inp.cache
+    gains = tile_gain(8)
+    kc = c.k_cache.float()
+    for b, L in enumerate(ctx):  # scale each cached key by the tile of its logical position
+        for p in range(L):
+            kc[int(c.block_table[b, p // 16]), p % 16] *= gains[p // TILE]
+    cache = inputs.PagedInputs(q=c.q, k_cache=kc.to(torch.bfloat16), v_cache=c.v_cache, block_table=c.block_table,
+                               seq_lens=c.seq_lens, block_size=c.block_size)
+    q = quiet_odd_rows(inp.q)
+    inp = inputs.ChunkedInputs(q=q, cu_q=inp.cu_q, cache=cache)
+    # sequence 0 seen as a dense problem: T = 600 new rows over S = 900 keys
+    k0 = torch.stack([cache.k_cache[int(c.block_table[0, p // 16]), p % 16, 0] for p in range(ctx[0])])
+    rows, mixed = rescale_events(f64(q[:ql[0], 0]), f64(k0), 0.3, True)
+    assert rows > 100 and mixed > 5
+    o, lse = run_chunked(inp, True, 0.3)
+    O, L = oracle_chunked(inp, True, 0.3)
+    check_close(f64(o), O, lse.numpy(), L, what="chunked rising")

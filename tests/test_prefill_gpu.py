@@ -76,3 +76,14 @@ def test_long_prefill_workload_sampled_rows():
     O, L = oracle_prefill(q, k, v, True, spec.scale, rows=rows)
     check_close(f64(o)[:, rows], O[:, rows], lse.numpy()[:, :, rows], L[:, :, rows], what="long_prefill rows")
     assert torch.isfinite(o.float()).all()
+
+
+def test_long_prefill_workload_all_rows():
+    """T = S = 16384: every element of O and LSE (16384 rows x 32 heads)
+    against the oracle, evaluated head by head in worker processes."""
+    from tests._oracle_pool import attention_by_head
+    spec = inputs.WORKLOADS["long_prefill_16k"]
+    q, k, v = inputs.make_prefill(spec)
+    o, lse = run_prefill(q, k, v, True, spec.scale)
+    O, L = attention_by_head(f64(q), f64(k), f64(v), spec.scale, True)
+    check_close(f64(o), O, lse.numpy(), L, what="long_prefill all rows")

@@ -1,12 +1,15 @@
 """The torch custom-op wrappers: fake (meta) shapes on CPU, and on the GPU
-the same results as the direct binding, inside torch.compile without a
-graph break (aot_eager backend: no code generation around the ops)."""
+results that match the fp64 oracle and are identical to the direct
+binding's, inside torch.compile without a graph break (aot_eager backend:
+no code generation around the ops)."""
 
 import pytest
 import torch
 
 from flashattention_attention_attn_b200 import inputs
 import flashattention_attention_attn_b200.torch_ops  # noqa: F401  (registers torch.ops.fa_b200)
+from tests._parity import (check_close, f64, oracle_chunked, oracle_decode, oracle_decode_fp8, oracle_prefill,
+                           oracle_varlen)
 
 
 def test_fake_shapes_without_running_anything():
@@ -37,7 +40,7 @@ def test_fake_shapes_without_running_anything():
 
 
 @pytest.mark.gpu
-def test_ops_match_binding_and_compile_without_graph_break():
+def test_ops_match_the_oracle_and_compile_without_graph_break():
     import flashattention_attention_attn_b200 as fa
     ps = inputs.PrefillSpec(B=1, Hq=8, Hkv=2, T=200, S=200, d=128, causal=True, seed=60)
     q, k, v = [t.cuda() for t in inputs.make_prefill(ps)]
@@ -60,10 +63,14 @@ def test_ops_match_binding_and_compile_without_graph_break():
     o, lse, od = g(q, k, v, dq, kc, vc, bt, sl)
     torch.cuda.synchronize()
     assert torch.equal(o, o_ref) and torch.equal(lse, lse_ref) and torch.equal(od, od_ref)
+    O, L = oracle_prefill(q.cpu(), k.cpu(), v.cpu(), True, ps.scale)
+    check_close(f64(o), O, f64(lse), L, what="torch op attn_fwd")
+    Od, _ = oracle_decode(d)
+    check_close(f64(od), Od, what="torch op paged_attn_decode")
 
 
 @pytest.mark.gpu
-def test_packed_chunked_and_fp8_ops_match_the_binding():
+def test_packed_chunked_and_fp8_ops_match_the_oracle_and_the_binding():
     from tests._parity import run_chunked, run_decode_fp8, run_varlen
     vs = inputs.VarlenSpec(B=3, Hq=8, Hkv=2, d=128, len_lo=1, len_hi=1, causal=True, seed=62)
     vin = inputs.make_varlen(vs, q_lens=[5, 130, 300])
@@ -71,6 +78,8 @@ def test_packed_chunked_and_fp8_ops_match_the_binding():
     o, lse = torch.ops.fa_b200.attn_fwd_varlen(vin.q.cuda(), vin.k.cuda(), vin.v.cuda(), vin.cu_q.cuda(),
                                                vin.cu_k.cuda(), vin.max_q, True, vs.scale)
     assert torch.equal(o.cpu(), o_ref) and torch.equal(lse.cpu(), lse_ref)
+    O, L = oracle_varlen(vin, True, vs.scale)
+    check_close(f64(o), O, f64(lse), L, what="torch op attn_fwd_varlen")
 
     cs = inputs.ChunkedSpec(B=2, Hq=8, Hkv=2, d=128, block_size=16, max_blocks=32, ctx_lo=1, ctx_hi=1, q_lo=1, q_hi=1,
                             seed=63)
@@ -81,6 +90,8 @@ def test_packed_chunked_and_fp8_ops_match_the_binding():
                                                   c.block_table.cuda(), c.seq_lens.cuda(), cin.cu_q.cuda(),
                                                   cin.max_q, True, cs.scale)
     assert torch.equal(o.cpu(), o_ref) and torch.equal(lse.cpu(), lse_ref)
+    O, L = oracle_chunked(cin, True, cs.scale)
+    check_close(f64(o), O, f64(lse), L, what="torch op paged_attn_prefill")
 
     ds = inputs.DecodeSpec(B=3, Hq=32, Hkv=8, d=128, block_size=16, max_blocks=16, ctx_lo=10, ctx_hi=250, seed=64)
     din = inputs.make_paged_fp8(ds)
@@ -89,3 +100,4 @@ def test_packed_chunked_and_fp8_ops_match_the_binding():
                                                  din.block_table.cuda(), din.seq_lens.cuda(), 0, din.k_scale,
                                                  din.v_scale)
     assert torch.equal(od.cpu(), od_ref)
+    check_close(f64(od), oracle_decode_fp8(din)[0], what="torch op paged_attn_decode_fp8")
