@@ -1,33 +1,36 @@
 """Benchmark of the fused-attention hot path on B200.
 
-One step = one pass of the whole path over one batch of synthetic input:
-  * attn_fwd          Llama3-8B-shaped causal GQA prefill (B=2, Hq=32, Hkv=8,
-                      T=S=512, d=128)
-  * paged_attn_decode one-token decode of 64 sequences against a paged cache
-                      (Hq=32, Hkv=8, d=128, block_size=16, context U[256,4096])
+One step = one pass of the whole path over one batch of synthetic input: a
+causal GQA prefill and a one-token paged-KV decode.  The default step is the
+long-context pair:
+  * attn_fwd          causal GQA prefill, B=1, Hq=32, Hkv=8, T=S=16384, d=128
+  * paged_attn_decode one-token decode of a 131072-token context through the
+                      block table (8192 permuted 16-token blocks), split-KV
 The metric is the fraction of the B200 roofline the step reaches: the ideal
 step time is prefill FLOPs / measured bf16 tensor peak + decode bytes /
 measured HBM bandwidth, and value = 100 * (sum over ranks of ideal time) /
 (measured step time, max over ranks): percent of one B200's roofline,
-summed over the GPUs of the job.
+summed over the GPUs of the job.  Each op is also timed alone (`parts`), and
+`roofline` reports the dominant one (the prefill) against its own peak.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                    [--workload step|long|varlen|chunked|fp8]
+                    [--workload long|step|varlen|chunked|fp8]
 
-`--workload long` times the long-context pair (T=S=16384 prefill and a
-131072-token split-KV decode) with the same accounting; `--workload varlen`
-replaces the prefill by 16 packed sequences of U[64, 2048] tokens
+`--workload step` times the Llama3-8B-shaped pair (T=S=512 prefill, B=2,
+and a 64-sequence decode with contexts of 256-4096 tokens); `--workload
+varlen` replaces that prefill by 16 packed sequences of U[64, 2048] tokens
 (attn_fwd_varlen); `--workload chunked` by a 512-token chunk of each of 8
 sequences against their paged cache of 1k-8k tokens (paged_attn_prefill);
-`--workload fp8` keeps the step but stores the decode cache as FP8 e4m3
-(paged_attn_decode_fp8; decode bytes count 1 byte per cached element).  `--impl reference`
-times the fp64 CPU oracle (the only reference implementation there is) on a
-bounded sample of the same step.
+`--workload fp8` keeps the Llama3-8B step but stores the decode cache as FP8
+e4m3 (paged_attn_decode_fp8; decode bytes count 1 byte per cached element).
+`--impl reference` times the fp64 CPU oracle (the only reference
+implementation there is) on a bounded sample of the same step.
 """
 
 from __future__ import annotations
 
 import argparse
+import hashlib
 import json
 import os
 import sys
@@ -38,34 +41,51 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 METRIC = "prefill attn TFLOP/s & paged-decode KV GB/s, % of B200 roofline"
-PART_TIMING = ("CUDA events around each part, on the launching stream, in a second K-step loop "
-               "run right after the timed one")
 UNIT = "% of 1xB200 roofline (summed over GPUs)"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+PART_TIMING = ("each op alone: K back-to-back calls on the launching stream, CUDA events at the two ends, "
+               "right after the timed step loop")
 
 WORKLOAD_SETS = {
-    "step": ("llama3_8b_prefill", "paged_decode_b64"),
     "long": ("long_prefill_16k", "long_decode_131k"),
+    "step": ("llama3_8b_prefill", "paged_decode_b64"),
     "varlen": ("varlen_prefill_16seq", "paged_decode_b64"),
     "chunked": ("chunked_prefill_paged", "paged_decode_b64"),
     "fp8": ("llama3_8b_prefill", "paged_decode_b64:fp8"),
 }
+DEFAULT_WORKLOAD = "long"
 
-
-# DRAM bytes (read + write) per launch of the dominant kernel of each step,
-# from the one-pass ncu launch lists of the same command (`dram__bytes_read.sum`
-# + `dram__bytes_write.sum`, mean over the captured launches), summarised in
-# profiles/launches_<workload>.md.  A value is dropped (None) whenever the
-# kernel changes after its capture.
-#   step / fp8: decode split kernel + LSE combine of one paged_attn_decode call
-#   long, varlen, chunked: the prefill launch
-TRAFFIC_BYTES = {
-    "step": 597.38e6 + 3.14e6 + 4.58e6,   # profiles/launches_llama3_8b_prefill_paged_decode_b64.md
-    "fp8": 299.00e6 + 2.79e6 + 4.58e6,    # profiles/launches_llama3_8b_prefill_paged_decode_b64_fp8.md
-    "long": 385.56e6 + 101.25e6,          # profiles/launches_long_prefill_16k_long_decode_131k.md
-    "varlen": 247.64e6 + 89.08e6,         # profiles/launches_varlen_prefill_16seq_paged_decode_b64.md
-    "chunked": 337.31e6 + 24.55e6,        # profiles/launches_chunked_prefill_paged_paged_decode_b64.md
+# DRAM bytes (read + write) per launch of each kernel of a step, from a
+# one-pass ncu launch list of `bench.py --workload <set>` (dram__bytes_read.sum
+# + dram__bytes_write.sum, mean over the captured launches of each kernel).
+# `csrc` is the source hash (csrc_hash() below) of the kernels that were
+# captured: when the kernels change, the figure no longer applies and the
+# bench reports null until a new capture replaces it.
+TRAFFIC = {
+    # set: {"prefill": bytes per launch, "decode": bytes per call (split + combine), "csrc": hash}
 }
+
+
+def csrc_hash() -> str:
+    """Hash of the CUDA sources (csrc/*.cu, *.cuh) the library is built from."""
+    d = os.path.join(ROOT, "flashattention_attention_attn_b200", "csrc")
+    h = hashlib.sha256()
+    for n in sorted(os.listdir(d)):
+        if n.endswith((".cu", ".cuh")):
+            h.update(n.encode())
+            with open(os.path.join(d, n), "rb") as f:
+                h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def traffic_of(workload: str, part: str):
+    """(bytes, note) for a kernel of a workload set, or (None, why not)."""
+    t = TRAFFIC.get(workload)
+    if not t or part not in t:
+        return None, "no ncu capture of this workload"
+    if t.get("csrc") != csrc_hash():
+        return None, "kernels changed since the ncu capture"
+    return t[part], "ncu DRAM read + write per launch, source hash %s" % t["csrc"]
 
 
 def decode_workload(dname):
@@ -74,11 +94,26 @@ def decode_workload(dname):
     return base, kind == "fp8"
 
 
+def vars_of(spec):
+    return {k: getattr(spec, k) for k in spec.__dataclass_fields__ if not k.startswith("_")}
+
+
+def step_config(pname, dname, inputs, world, args, prefill_in_bytes, decode_bytes):
+    """The `config` object of the JSON line; identical for both --impl arms."""
+    pspec = (inputs.VARLEN_WORKLOADS.get(pname) or inputs.CHUNKED_WORKLOADS.get(pname) or inputs.WORKLOADS[pname])
+    dbase, dfp8 = decode_workload(dname)
+    return {"workload": f"{pname} + {dname}", "prefill": vars_of(pspec),
+            "decode": {**vars_of(inputs.WORKLOADS[dbase]), "kv_cache": "fp8 e4m3" if dfp8 else "bf16"},
+            "decode_num_splits": args.num_splits or "auto", "parallelism": f"replicas x{world} (no exchange)",
+            "streams": ("prefill and decode concurrently on two streams (fork/join every step)"
+                        if args.streams == 2 else "prefill then decode on one stream"),
+            "l2": ("no flush between steps; per step the prefill moves %.0f MB (inputs read once, outputs written "
+                   "once) and the decode reads %.0f MB (L2: 126 MB)" % (prefill_in_bytes / 1e6, decode_bytes / 1e6))}
+
+
 class PrefillCase:
-    """The prefill half of a step: dense (attn_fwd) or packed (attn_fwd_varlen); `--workload chunked` by a 512-token chunk of each of 8
-sequences against their paged cache of 1k-8k tokens (paged_attn_prefill);
-`--workload fp8` keeps the step but stores the decode cache as FP8 e4m3
-(paged_attn_decode_fp8; decode bytes count 1 byte per cached element)."""
+    """The prefill half of a step: dense (attn_fwd), packed (attn_fwd_varlen)
+    or chunked against a paged cache (paged_attn_prefill)."""
 
     def __init__(self, name, seed, dev, fa, inputs, workloads):
         import torch
@@ -98,7 +133,6 @@ sequences against their paged cache of 1k-8k tokens (paged_attn_prefill);
             self.dev_in = [t.to(dev) for t in self.host_in]
             self.o = torch.empty_like(self.dev_in[0])
             self.lse = torch.empty(sp.Hq, self.total_q, device=dev, dtype=torch.float32)
-            self.config = {**vars_of(sp), "context_lengths": ctx, "query_counts": lens_q}
         elif self.varlen:
             sp = self.spec = inputs.VARLEN_WORKLOADS[name]
             vin = inputs.make_varlen(sp, seed=seed)
@@ -112,7 +146,6 @@ sequences against their paged cache of 1k-8k tokens (paged_attn_prefill);
             self.dev_in = [t.to(dev) for t in self.host_in]
             self.o = torch.empty_like(self.dev_in[0])
             self.lse = torch.empty(sp.Hq, self.total_q, device=dev, dtype=torch.float32)
-            self.config = {**vars_of(sp), "lengths": lens_q, "total_tokens": self.total_q}
         else:
             sp = self.spec = inputs.WORKLOADS[name]
             q, k, v = inputs.make_prefill(sp, seed=seed)
@@ -122,7 +155,6 @@ sequences against their paged cache of 1k-8k tokens (paged_attn_prefill);
             self.dev_in = [t.to(dev) for t in self.host_in]
             self.o = torch.empty_like(self.dev_in[0])
             self.lse = torch.empty(sp.B, sp.Hq, sp.T, device=dev, dtype=torch.float32)
-            self.config = vars_of(sp)
         self.fa = fa
 
     def call(self, stream):
@@ -154,10 +186,10 @@ def load_peaks():
 def parse_args(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=2000)
-    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--steps", type=int, default=100)
+    ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", choices=sorted(WORKLOAD_SETS), default="step")
+    ap.add_argument("--workload", choices=sorted(WORKLOAD_SETS), default=DEFAULT_WORKLOAD)
     ap.add_argument("--num-splits", type=int, default=0, help="decode splits (0 = library's choice)")
     ap.add_argument("--e2e-steps", type=int, default=5)
     ap.add_argument("--streams", type=int, choices=[1, 2], default=2,
@@ -167,22 +199,23 @@ def parse_args(argv=None):
 
 
 # --------------------------------------------------------------------------
-# clocks during the timed region (NVML reads only; nothing is changed)
+# clocks during the timed regions (NVML reads only; nothing is changed)
 # --------------------------------------------------------------------------
 class ClockSampler:
-    """Samples SM clock and clock-event reasons every 20 ms from an
-    `nvidia-smi -lms` child process (independent of this process's GIL), with
-    NVML polling in a thread as the fallback.  Each sample is stamped with
-    time.perf_counter() when it arrives."""
+    """Samples the SM clock and the clock-event reasons of one GPU every
+    `period_s` through NVML, from a thread (NVML calls release the GIL), each
+    sample stamped with time.perf_counter().  `summary(t0, t1)` reports the
+    samples inside a window.  `nvidia-smi -lms` is the fallback when NVML
+    cannot be used."""
     REASONS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
                0x8: "hw_slowdown", 0x10: "sync_boost", 0x20: "sw_thermal_slowdown",
                0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown", 0x100: "display_clock_setting"}
 
-    def __init__(self, device_index: int, period_s: float = 0.02):
+    def __init__(self, device_index: int, period_s: float = 0.002):
         self.samples = []
         self.period = period_s
-        # nvidia-smi and NVML number GPUs physically; CUDA_VISIBLE_DEVICES may
-        # not, so the device is named by its UUID when torch reports one.
+        # NVML numbers GPUs physically; CUDA_VISIBLE_DEVICES may not, so the
+        # device is named by its UUID when torch reports one.
         self.ident = str(device_index)
         try:
             import torch
@@ -204,8 +237,21 @@ class ClockSampler:
             self._h = (pynvml.nvmlDeviceGetHandleByUUID(self.ident.encode()) if self.ident.startswith("GPU-")
                        else pynvml.nvmlDeviceGetHandleByIndex(device_index))
             self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
+            self._reasons = getattr(pynvml, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+                pynvml.nvmlDeviceGetCurrentClocksThrottleReasons
         except Exception:
             self._nv = None
+
+    def _poll_nvml(self):
+        nv = self._nv
+        while not self._stop.is_set():
+            try:
+                mhz = nv.nvmlDeviceGetClockInfo(self._h, nv.NVML_CLOCK_SM)
+                rs = self._reasons(self._h)
+                self.samples.append((time.perf_counter(), mhz, rs))
+            except Exception:
+                pass
+            time.sleep(self.period)
 
     def _read_smi(self):
         for line in self._proc.stdout:
@@ -217,37 +263,27 @@ class ClockSampler:
             except (ValueError, IndexError):
                 pass
 
-    def _poll_nvml(self):
-        nv = self._nv
-        while not self._stop.is_set():
-            try:
-                mhz = nv.nvmlDeviceGetClockInfo(self._h, nv.NVML_CLOCK_SM)
-                rs = nv.nvmlDeviceGetCurrentClocksEventReasons(self._h)
-                self.samples.append((time.perf_counter(), mhz, rs))
-            except Exception:
-                pass
-            time.sleep(self.period)
-
     def start(self, wait_s: float = 5.0):
-        import shutil
-        import subprocess
-        smi = shutil.which("nvidia-smi")
-        if smi is not None:
-            try:
-                self._proc = subprocess.Popen(
-                    [smi, "-i", self.ident, "--query-gpu=clocks.sm,clocks.max.sm,clocks_event_reasons.active",
-                     "--format=csv,noheader,nounits", "-lms", str(int(self.period * 1000))],
-                    stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True, bufsize=1)
-                self._thr = threading.Thread(target=self._read_smi, daemon=True)
-                self.source = "nvidia-smi -lms %d" % int(self.period * 1000)
-            except OSError:
-                self._proc = None
-        if self._proc is None and self._nv is not None:
+        if self._nv is not None:
             self._thr = threading.Thread(target=self._poll_nvml, daemon=True)
-            self.source = "nvml polling"
+            self.source = "nvml polling every %g ms" % (self.period * 1000)
+        else:
+            import shutil
+            import subprocess
+            smi = shutil.which("nvidia-smi")
+            if smi is not None:
+                try:
+                    self._proc = subprocess.Popen(
+                        [smi, "-i", self.ident, "--query-gpu=clocks.sm,clocks.max.sm,clocks_event_reasons.active",
+                         "--format=csv,noheader,nounits", "-lms", "20"],
+                        stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True, bufsize=1)
+                    self._thr = threading.Thread(target=self._read_smi, daemon=True)
+                    self.source = "nvidia-smi -lms 20"
+                except OSError:
+                    self._proc = None
         if self._thr is not None:
             self._thr.start()
-            t_end = time.perf_counter() + wait_s  # the timed region starts once samples flow
+            t_end = time.perf_counter() + wait_s  # the timed regions start once samples flow
             while not self.samples and time.perf_counter() < t_end:
                 time.sleep(0.01)
 
@@ -277,107 +313,129 @@ class ClockSampler:
                 "source": self.source}
 
 
+def timed_region(torch, stream, body, K, sampler, world, dist):
+    """K calls of `body` with CUDA events on `stream` at the two ends only,
+    bracketed by a barrier and a device synchronisation on both sides.
+    Returns (milliseconds per call, clock summary of the region)."""
+    start = torch.cuda.Event(enable_timing=True)
+    end = torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    t0 = time.perf_counter()
+    start.record(stream)
+    for _ in range(K):
+        body()
+    end.record(stream)
+    while not end.query():  # the sampler thread records clocks meanwhile
+        time.sleep(0.0005)
+    torch.cuda.synchronize()
+    t1 = time.perf_counter()
+    if world > 1:
+        dist.barrier()
+    return start.elapsed_time(end) / K, sampler.summary(t0, t1)
+
+
 # --------------------------------------------------------------------------
 # CPU baseline: the fp64 oracle on a bounded sample of the same step
 # --------------------------------------------------------------------------
-def _cpu_prefill_dense(pname, seed_offset, orc, inputs, workloads, f):
-    """Oracle time of a dense prefill, from an evenly spread set of rows of
-    batch 0 (all heads), scaled by visible pairs to the whole workload."""
-    ps = inputs.WORKLOADS[pname]
-    q, k, v = inputs.make_prefill(ps, seed=ps.seed + seed_offset)
-    qd, kd, vd = f(q), f(k), f(v)
-    T = ps.T
-    rows = list(range(0, T, max(1, T // 64)))
-    t0 = time.perf_counter()
-    orc.attention(qd[:1], kd[:1], vd[:1], ps.scale, ps.causal, rows=rows)
-    tp = time.perf_counter() - t0
-    seen = sum(min(ps.S, i + ps.S - ps.T + 1) if ps.causal else ps.S for i in rows)  # cost ~ keys seen
-    full_pairs = workloads.visible_pairs(ps.T, ps.S, ps.causal) * ps.B
-    flops = workloads.prefill_flops(ps.B, ps.Hq, ps.T, ps.S, ps.d, ps.causal)
-    return tp * full_pairs / max(seen, 1), flops, f"rows {len(rows)}/{T} of batch 0 (all {ps.Hq} heads)"
+class CpuSample:
+    """The fp64 oracle on a bounded sample of one step's workloads.  The
+    inputs are drawn once; `run()` times the oracle on the sample and scales
+    that time to the whole step by visible (query, key) pairs for the
+    prefill and by cached tokens for the decode."""
 
+    def __init__(self, pname, dname, peaks, seed_offset=0, decode_budget_s=10.0):
+        import torch
 
-def _cpu_prefill_varlen(pname, seed_offset, orc, inputs, workloads, f):
-    """Oracle time of a packed prefill, from its first two sequences, scaled
-    by visible pairs to all sequences."""
-    sp = inputs.VARLEN_WORKLOADS[pname]
-    vin = inputs.make_varlen(sp, seed=sp.seed + seed_offset)
-    lq = (vin.cu_q[1:] - vin.cu_q[:-1]).tolist()
-    lk = (vin.cu_k[1:] - vin.cu_k[:-1]).tolist()
-    n = 2
-    cq, ck = vin.cu_q[:n + 1].numpy(), vin.cu_k[:n + 1].numpy()
-    t0 = time.perf_counter()
-    orc.attention_varlen(f(vin.q[:cq[-1]]), f(vin.k[:ck[-1]]), f(vin.v[:ck[-1]]), cq, ck, sp.scale, sp.causal)
-    tp = time.perf_counter() - t0
-    pairs = [workloads.visible_pairs(t, s_, sp.causal) for t, s_ in zip(lq, lk)]
-    flops = sum(workloads.prefill_flops(1, sp.Hq, t, s_, sp.d, sp.causal) for t, s_ in zip(lq, lk))
-    return tp * sum(pairs) / max(sum(pairs[:n]), 1), flops, f"sequences {n}/{sp.B} (all {sp.Hq} heads)"
+        from flashattention_attention_attn_b200 import inputs, workloads
+        from oracle import fp64_attention as orc
+        self.orc = orc
+        f = lambda t: t.to(torch.float64).numpy()  # noqa: E731
+        try:
+            from threadpoolctl import threadpool_info
+            self.cores = max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
+        except Exception:
+            self.cores = 1
+        self.decode_budget_s = decode_budget_s
+        if pname in inputs.VARLEN_WORKLOADS:
+            sp = inputs.VARLEN_WORKLOADS[pname]
+            vin = inputs.make_varlen(sp, seed=sp.seed + seed_offset)
+            lq = (vin.cu_q[1:] - vin.cu_q[:-1]).tolist()
+            lk = (vin.cu_k[1:] - vin.cu_k[:-1]).tolist()
+            n = 2
+            cq, ck = vin.cu_q[:n + 1].numpy(), vin.cu_k[:n + 1].numpy()
+            a = (f(vin.q[:cq[-1]]), f(vin.k[:ck[-1]]), f(vin.v[:ck[-1]]), cq, ck, sp.scale, sp.causal)
+            self.prefill_fn = lambda: orc.attention_varlen(*a)
+            pairs = [workloads.visible_pairs(t, s_, sp.causal) for t, s_ in zip(lq, lk)]
+            self.prefill_scale = sum(pairs) / max(sum(pairs[:n]), 1)
+            self.flops = sum(workloads.prefill_flops(1, sp.Hq, t, s_, sp.d, sp.causal) for t, s_ in zip(lq, lk))
+            self.pdesc = f"sequences {n}/{sp.B} (all {sp.Hq} heads), scaled by visible pairs"
+            self.prefill_bytes = sum(workloads.prefill_min_bytes(1, sp.Hq, sp.Hkv, t, s_, sp.d) for t, s_ in zip(lq, lk))
+        elif pname in inputs.CHUNKED_WORKLOADS:
+            sp = inputs.CHUNKED_WORKLOADS[pname]
+            ci = inputs.make_chunked(sp, seed=sp.seed + seed_offset)
+            c = ci.cache
+            lq = (ci.cu_q[1:] - ci.cu_q[:-1]).tolist()
+            ctx = c.seq_lens.tolist()
+            a = (f(ci.q[:lq[0]]), f(c.k_cache), f(c.v_cache), c.block_table.numpy()[:1], ctx[:1], ci.cu_q.numpy()[:2],
+                 c.block_size, sp.scale, sp.causal)
+            self.prefill_fn = lambda: orc.paged_prefill(*a)
+            pairs = [workloads.visible_pairs(t, s_, sp.causal) for t, s_ in zip(lq, ctx)]
+            self.prefill_scale = sum(pairs) / max(pairs[0], 1)
+            self.flops = sum(workloads.prefill_flops(1, sp.Hq, t, s_, sp.d, sp.causal) for t, s_ in zip(lq, ctx))
+            self.pdesc = f"sequences 1/{sp.B} (all {sp.Hq} heads), scaled by visible pairs"
+            self.prefill_bytes = sum(workloads.prefill_min_bytes(1, sp.Hq, sp.Hkv, t, s_, sp.d) for t, s_ in zip(lq, ctx))
+        else:
+            ps = inputs.WORKLOADS[pname]
+            q, k, v = inputs.make_prefill(ps, seed=ps.seed + seed_offset)
+            qd, kd, vd = f(q[:1]), f(k[:1]), f(v[:1])
+            rows = list(range(0, ps.T, max(1, ps.T // 64)))
+            self.prefill_fn = lambda: orc.attention(qd, kd, vd, ps.scale, ps.causal, rows=rows)
+            # the oracle forms every row's full score row, so its cost goes with the rows
+            self.prefill_scale = ps.B * ps.T / len(rows)
+            self.flops = workloads.prefill_flops(ps.B, ps.Hq, ps.T, ps.S, ps.d, ps.causal)
+            self.pdesc = f"rows {len(rows)}/{ps.T} of batch 0 (all {ps.Hq} heads), scaled by rows"
+            self.prefill_bytes = workloads.prefill_min_bytes(ps.B, ps.Hq, ps.Hkv, ps.T, ps.S, ps.d)
+        dbase, dfp8 = decode_workload(dname)
+        ds = inputs.WORKLOADS[dbase]
+        if dfp8:
+            dinp = inputs.make_paged_fp8(ds, seed=ds.seed + seed_offset)
+            self.kc = dinp.k_scale * orc.decode_e4m3(dinp.k_cache.numpy())
+            self.vc = dinp.v_scale * orc.decode_e4m3(dinp.v_cache.numpy())
+        else:
+            dinp = inputs.make_paged(ds, seed=ds.seed + seed_offset)
+            self.kc, self.vc = f(dinp.k_cache), f(dinp.v_cache)
+        self.ds, self.q, self.table = ds, f(dinp.q), dinp.block_table.numpy()
+        self.lens = dinp.seq_lens.numpy()
+        self.dbytes = workloads.decode_bytes(self.lens, ds.Hq, ds.Hkv, ds.d, ds.block_size,
+                                             kv_elem_bytes=1 if dfp8 else 2)
+        self.ideal = self.flops / (peaks["bf16_tflops"] * 1e12) + self.dbytes / (peaks["hbm_gbs"] * 1e9)
 
-
-def _cpu_prefill_chunked(pname, seed_offset, orc, inputs, workloads, f):
-    """Oracle time of a chunked paged prefill, from its first sequence,
-    scaled by visible pairs to all sequences."""
-    sp = inputs.CHUNKED_WORKLOADS[pname]
-    ci = inputs.make_chunked(sp, seed=sp.seed + seed_offset)
-    c = ci.cache
-    lq = (ci.cu_q[1:] - ci.cu_q[:-1]).tolist()
-    ctx = c.seq_lens.tolist()
-    t0 = time.perf_counter()
-    orc.paged_prefill(f(ci.q[:lq[0]]), f(c.k_cache), f(c.v_cache), c.block_table.numpy()[:1], ctx[:1],
-                      ci.cu_q.numpy()[:2], c.block_size, sp.scale, sp.causal)
-    tp = time.perf_counter() - t0
-    pairs = [workloads.visible_pairs(t, s_, sp.causal) for t, s_ in zip(lq, ctx)]
-    flops = sum(workloads.prefill_flops(1, sp.Hq, t, s_, sp.d, sp.causal) for t, s_ in zip(lq, ctx))
-    return tp * sum(pairs) / max(pairs[0], 1), flops, f"sequences 1/{sp.B} (all {sp.Hq} heads)"
-
-
-def cpu_baseline(pname, dname, peaks, seed_offset=0, budget_s=20.0):
-    import torch
-
-    from flashattention_attention_attn_b200 import inputs, workloads
-    from oracle import fp64_attention as orc
-
-    try:
-        from threadpoolctl import threadpool_info
-        cores = max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
-    except Exception:
-        cores = 1
-    f = lambda t: t.to(torch.float64).numpy()  # noqa: E731
-    if pname in inputs.VARLEN_WORKLOADS:
-        t_prefill, flops, pdesc = _cpu_prefill_varlen(pname, seed_offset, orc, inputs, workloads, f)
-    elif pname in inputs.CHUNKED_WORKLOADS:
-        t_prefill, flops, pdesc = _cpu_prefill_chunked(pname, seed_offset, orc, inputs, workloads, f)
-    else:
-        t_prefill, flops, pdesc = _cpu_prefill_dense(pname, seed_offset, orc, inputs, workloads, f)
-    dbase, dfp8 = decode_workload(dname)
-    ds = inputs.WORKLOADS[dbase]
-    if dfp8:
-        dinp = inputs.make_paged_fp8(ds, seed=ds.seed + seed_offset)
-        kc = dinp.k_scale * orc.decode_e4m3(dinp.k_cache.numpy())
-        vc = dinp.v_scale * orc.decode_e4m3(dinp.v_cache.numpy())
-    else:
-        dinp = inputs.make_paged(ds, seed=ds.seed + seed_offset)
-        kc, vc = f(dinp.k_cache), f(dinp.v_cache)
-    # decode sample: leading sequences until ~budget/2 spent or 4 sequences
-    lens = dinp.seq_lens.numpy()
-    qq = f(dinp.q)
-    done_tok, td, nseq = 0, 0.0, 0
-    for b in range(len(lens)):
+    def run(self):
+        """Oracle seconds for the whole step, estimated from the sample."""
         t0 = time.perf_counter()
-        orc.paged_decode(qq[b:b + 1], kc, vc, dinp.block_table.numpy()[b:b + 1], lens[b:b + 1], 16, ds.scale)
-        td += time.perf_counter() - t0
-        done_tok += int(lens[b])
-        nseq += 1
-        if nseq >= 4 or td > budget_s / 2:
-            break
-    t_decode = td * float(lens.sum()) / max(done_tok, 1)
-    dbytes = workloads.decode_bytes(lens, ds.Hq, ds.Hkv, ds.d, ds.block_size, kv_elem_bytes=1 if dfp8 else 2)
-    ideal = flops / (peaks["bf16_tflops"] * 1e12) + dbytes / (peaks["hbm_gbs"] * 1e9)
-    est = t_prefill + t_decode
-    return {"value": 100.0 * ideal / est, "unit": UNIT, "cores": int(cores), "kind": "oracle",
-            "sample": (f"fp64 oracle: prefill {pdesc}, decode {nseq}/{len(lens)} sequences ({done_tok} tokens); "
-                       f"time scaled by visible pairs / tokens to the full step"),
-            "est_step_s": est}
+        self.prefill_fn()
+        t_prefill = (time.perf_counter() - t0) * self.prefill_scale
+        done_tok, td, nseq = 0, 0.0, 0
+        for b in range(len(self.lens)):  # leading sequences, until the budget or 4 sequences
+            t0 = time.perf_counter()
+            self.orc.paged_decode(self.q[b:b + 1], self.kc, self.vc, self.table[b:b + 1], self.lens[b:b + 1],
+                                  self.ds.block_size, self.ds.scale)
+            td += time.perf_counter() - t0
+            done_tok += int(self.lens[b])
+            nseq += 1
+            if nseq >= 4 or td > self.decode_budget_s:
+                break
+        t_decode = td * float(self.lens.sum()) / max(done_tok, 1)
+        self.sample = (f"fp64 oracle: prefill {self.pdesc}, decode {nseq}/{len(self.lens)} sequences "
+                       f"({done_tok} tokens), scaled by tokens; the sum estimates the whole step")
+        return t_prefill + t_decode
+
+    def baseline(self):
+        est = self.run()
+        return {"value": 100.0 * self.ideal / est, "unit": UNIT, "cores": int(self.cores), "kind": "oracle",
+                "sample": self.sample}
 
 
 # --------------------------------------------------------------------------
@@ -429,9 +487,7 @@ def main():
     # --streams 2 they run concurrently: the prefill on the current stream,
     # the decode on a second stream of the same priority that forks from it
     # and joins it again every step, so the decode's CTAs fill the SMs the
-    # prefill leaves idle.  All timing events sit on the current stream.  (A
-    # higher priority for the prefill's stream measured slower on the default
-    # and FP8 steps.)
+    # prefill leaves idle.  All timing events sit on the current stream.
     stream = torch.cuda.current_stream(dev)
     side = torch.cuda.Stream(dev) if args.streams == 2 else stream
     fork_ev, join_ev = torch.cuda.Event(), torch.cuda.Event()
@@ -466,46 +522,20 @@ def main():
     torch.cuda.synchronize()
 
     K = args.steps
-    start = torch.cuda.Event(enable_timing=True)
-    end = torch.cuda.Event(enable_timing=True)
     sampler = ClockSampler(local_rank)
     sampler.start()
-    time.sleep(0.05)
-    if world > 1:
-        dist.barrier()
-    torch.cuda.synchronize()
-    t_wall0 = time.perf_counter()
-    # Only the two ends are recorded: an event between two kernels would cut
-    # the programmatic overlap of one kernel's prologue with the previous tail.
-    start.record(stream)
-    for i in range(K):
-        step()
-    end.record(stream)
-    torch.cuda.synchronize()
-    t_wall1 = time.perf_counter()
-    if world > 1:
-        dist.barrier()
+    # The timed step loop (the value).  Only its two ends are recorded: an
+    # event between two kernels would cut the programmatic overlap of one
+    # kernel's prologue with the previous one's tail.
+    ms_step, clocks = timed_region(torch, stream, step, K, sampler, world, dist)
+    # Each op alone, K back-to-back calls (the per-op roofline fractions).
+    ms_pre, clocks_pre = timed_region(torch, stream, lambda: pre.call(stream), K, sampler, world, dist)
+    ms_dec, clocks_dec = timed_region(torch, stream, lambda: decode_call(stream), K, sampler, world, dist)
     sampler.stop()
-    total_ms = start.elapsed_time(end)
-
-    # Per-part split (reported, not the value): K more steps with events
-    # between the parts, both parts on one stream.
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(K)]
-    for i in range(K):
-        ev[i][0].record(stream)
-        pre.call(stream)
-        ev[i][1].record(stream)
-        decode_call(stream)
-        ev[i][2].record(stream)
-    torch.cuda.synchronize()
     status = fa.attn_read_device_status(clear=True)
     if status != 0:
         raise RuntimeError(f"device status {status}: a bounded wait timed out")
-
-    t_pre = sum(ev[i][0].elapsed_time(ev[i][1]) for i in range(K)) / K
-    t_dec = sum(ev[i][1].elapsed_time(ev[i][2]) for i in range(K)) / K
-    ms_step = total_ms / K
-    ms_step, t_pre, t_dec = dist_util.max_over_ranks([ms_step, t_pre, t_dec], device=dev)
+    ms_step, ms_pre, ms_dec = dist_util.max_over_ranks([ms_step, ms_pre, ms_dec], device=dev)
 
     ideal_pre = flops / (peaks["bf16_tflops"] * 1e12)
     ideal_dec = dbytes / (peaks["hbm_gbs"] * 1e9)
@@ -551,83 +581,69 @@ def main():
     if rank != 0:
         return 0
 
-    dec_gbs = dbytes / (t_dec * 1e-3) / 1e9
-    pre_tflops = flops / (t_pre * 1e-3) / 1e12
-    clocks = sampler.summary(t_wall0, t_wall1)
-    dominant = "decode" if t_dec >= t_pre else "prefill"
-    if dominant == "decode":
-        roofline = {"bound": "hbm", "achieved": dec_gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                    "frac": dec_gbs / peaks["hbm_gbs"], "traffic": TRAFFIC_BYTES.get(args.workload),
-                    "traffic_unit": "bytes per call (ncu DRAM read + write)", "algorithmic_bytes": dbytes,
-                    "kernel": "paged_attn_decode (split kernel + LSE combine)",
-                    "peak_source": f"{peak_src} (hbm_gbs)", "duration": PART_TIMING}
-    else:
-        # The burst GEMM peak applies to a kernel that runs in short bursts; if
-        # the power cap was active during the timed loop, the sustained one.
-        capped = "sw_power_cap" in clocks.get("reasons", [])
-        tpeak = peaks["bf16_tflops_sustained"] if capped else peaks["bf16_tflops"]
+    dec_gbs = dbytes / (ms_dec * 1e-3) / 1e9
+    pre_tflops = flops / (ms_pre * 1e-3) / 1e12
+    # The burst GEMM peak applies to a kernel timed in short bursts; if the
+    # power cap was active while it was timed, the sustained one.
+    capped = "sw_power_cap" in clocks_pre.get("reasons", [])
+    tpeak = peaks["bf16_tflops_sustained"] if capped else peaks["bf16_tflops"]
+    tpeak_src = (f"{peak_src} (bf16_tflops_sustained: sw_power_cap active while the prefill was timed)"
+                 if capped else f"{peak_src} (bf16_tflops, burst)")
+    pre_traffic, pre_tnote = traffic_of(args.workload, "prefill")
+    dec_traffic, dec_tnote = traffic_of(args.workload, "decode")
+    parts = {
+        "prefill": {"op": pre.name, "ms": ms_pre, "tflops": pre_tflops, "peak": tpeak, "frac": pre_tflops / tpeak,
+                    "peak_source": tpeak_src, "flops": flops, "algorithmic_bytes": pre.min_bytes,
+                    "traffic": pre_traffic, "traffic_note": pre_tnote, "clocks": clocks_pre},
+        "decode": {"op": dname, "ms": ms_dec, "gbs": dec_gbs, "peak": peaks["hbm_gbs"],
+                   "frac": dec_gbs / peaks["hbm_gbs"], "peak_source": f"{peak_src} (hbm_gbs)", "bytes": dbytes,
+                   "traffic": dec_traffic, "traffic_note": dec_tnote, "clocks": clocks_dec},
+    }
+    if ms_pre >= ms_dec:  # the op that takes longer alone
         roofline = {"bound": "tensor", "achieved": pre_tflops, "peak": tpeak, "unit": "TFLOP/s",
-                    "frac": pre_tflops / tpeak, "traffic": TRAFFIC_BYTES.get(args.workload),
-                    "traffic_unit": "bytes per launch (ncu DRAM read + write)", "algorithmic_bytes": pre.min_bytes,
-                    "kernel": "attn_fwd",
-                    "peak_source": (f"{peak_src} (bf16_tflops_sustained: sw_power_cap active in the timed loop)"
-                                    if capped else f"{peak_src} (bf16_tflops, burst)"),
-                    "duration": PART_TIMING}
-    launches_per_step = 1 + 1 + 1  # prefill, decode split kernel, LSE combine
+                    "frac": pre_tflops / tpeak, "traffic": pre_traffic, "traffic_note": pre_tnote,
+                    "algorithmic_bytes": pre.min_bytes, "kernel": f"prefill ({pre.name})",
+                    "peak_source": tpeak_src, "duration": PART_TIMING}
+    else:
+        roofline = {"bound": "hbm", "achieved": dec_gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                    "frac": dec_gbs / peaks["hbm_gbs"], "traffic": dec_traffic, "traffic_note": dec_tnote,
+                    "algorithmic_bytes": dbytes, "kernel": f"paged decode ({dname}; split kernel + LSE combine)",
+                    "peak_source": f"{peak_src} (hbm_gbs)", "duration": PART_TIMING}
+    combine = 1 if (splits != 1) else 0  # the LSE combine runs whenever the decode uses more than one split
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K, "warmup": args.warmup,
         "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "bf16", "data": "synthetic (seeded N(0,1) bf16; random block-id permutations)",
-        "config": {"workload": f"{pname} + {dname}", "prefill": pre.config,
-                   "decode": {**vars_of(ds), "kv_cache": "fp8 e4m3" if dfp8 else "bf16"},
-                   "decode_num_splits": splits or "auto", "parallelism": f"replicas x{world} (no exchange)",
-                   "streams": ("prefill and decode concurrently on two streams (fork/join every step)"
-                               if args.streams == 2 else "prefill then decode on one stream"),
-                   "l2": "inputs larger than L2 (decode KV cache %.0f MB per step)" % (dbytes / 1e6)},
-        "parts": {"prefill": {"ms": t_pre, "tflops": pre_tflops, "frac": pre_tflops / peaks["bf16_tflops"],
-                              "flops": flops},
-                  "decode": {"ms": t_dec, "gbs": dec_gbs, "frac": dec_gbs / peaks["hbm_gbs"],
-                             "bytes": dbytes}},
+        "config": step_config(pname, dname, inputs, world, args, pre.min_bytes, dbytes),
+        "parts": parts,
         "roofline": roofline,
         "e2e": e2e,
-        "gpu_launches": launches_per_step * K,
+        "gpu_launches": (2 + combine) * K,
         "clocks": clocks,
         "peaks": {**peaks, "source": peak_src},
+        "csrc_hash": csrc_hash(),
     }
     if not args.no_cpu_baseline and world == 1:
-        cb = cpu_baseline(pname, dname, peaks)
-        cb.pop("est_step_s", None)
-        line["cpu_baseline"] = cb
+        line["cpu_baseline"] = CpuSample(pname, dname, peaks).baseline()
     print(json.dumps(line))
     return 0
 
 
-def vars_of(spec):
-    return {k: getattr(spec, k) for k in spec.__dataclass_fields__ if not k.startswith("_")}
-
-
 def run_reference(args, pname, dname, peaks, peak_src, world):
     """The fp64 CPU oracle, each step a bounded sample of the same workload."""
-    steps = []
-    info = None
-    for i in range(max(0, args.warmup) + args.steps):
-        budget = 20.0 / max(1, args.steps)
-        r = cpu_baseline(pname, dname, peaks, budget_s=budget)
-        if i >= args.warmup:
-            steps.append(r["est_step_s"])
-            info = r
-    est = sum(steps) / len(steps)
     from flashattention_attention_attn_b200 import inputs
-    value = info["value"]
+    budget = max(0.5, 10.0 / max(1, args.steps))  # decode seconds per step: the run stays within minutes
+    cs = CpuSample(pname, dname, peaks, decode_budget_s=budget)
+    for _ in range(max(0, args.warmup)):
+        cs.run()
+    est = sum(cs.run() for _ in range(args.steps)) / max(1, args.steps)
+    value = 100.0 * cs.ideal / est
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": est * 1e3, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic (same seeds as ours)",
-        "config": {"workload": f"{pname} + {dname}", "prefill": vars_of(inputs.VARLEN_WORKLOADS.get(pname) or inputs.CHUNKED_WORKLOADS.get(pname)
-                                     or inputs.WORKLOADS[pname]),
-                   "decode": vars_of(inputs.WORKLOADS[decode_workload(dname)[0]])},
-        "cpu_baseline": {"value": value, "unit": UNIT, "cores": info["cores"], "kind": "oracle",
-                         "sample": info["sample"]},
+        "config": step_config(pname, dname, inputs, world, args, cs.prefill_bytes, cs.dbytes),
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": cs.cores, "kind": "oracle", "sample": cs.sample},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
         "peaks": {**peaks, "source": peak_src},
     }
