@@ -55,9 +55,10 @@ def test_product_path_does_not_use_the_oracle_or_triton():
     bad = [p for p in product if imp.search(_read(p))]
     assert not bad, bad
     # bench.py reaches the oracle only from its CPU-baseline / reference leg
+    # (the CpuSample class, which both use)
     bench = _read(os.path.join(ROOT, "bench.py"))
     for m in re.finditer(r"^\s*(from oracle|import oracle)", bench, re.M):
         line = bench[: m.start()].count("\n") + 1
-        head = bench[: m.start()]
-        fn = head[head.rfind("\ndef ") + 1:].split("(", 1)[0]
-        assert fn in ("def cpu_baseline", "def run_reference"), (line, fn)
+        # the enclosing top-level definition (a line that starts in column 0)
+        tops = re.findall(r"^(def \w+|class \w+)", bench[: m.start()], re.M)
+        assert tops and tops[-1] in ("class CpuSample", "def run_reference"), (line, tops[-1:])
