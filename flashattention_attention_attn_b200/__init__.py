@@ -15,8 +15,10 @@ call does, and raises if it is missing.
 from . import inputs  # noqa: F401  (seeded synthetic inputs; no arithmetic)
 
 _BINDING_NAMES = {
-    "attn_fwd", "attn_fwd_varlen", "paged_attn_decode", "paged_attn_decode_fp8", "paged_attn_decode_noalloc", "paged_attn_prefill", "attn_check_support", "attn_status_string",
-    "attn_read_device_status", "attn_selftest_bounded_wait", "library", "library_path", "AttnError",
+    "attn_fwd", "attn_fwd_varlen", "paged_attn_decode", "paged_attn_decode_fp8", "paged_attn_decode_noalloc",
+    "paged_attn_prefill", "paged_attn_decode_checked", "paged_attn_decode_fp8_checked", "paged_attn_prefill_checked",
+    "attn_check_support", "attn_status_string", "attn_read_device_status", "attn_selftest_bounded_wait", "library",
+    "library_path", "AttnError", "ATTN_DEVSTATUS_TIMEOUT", "ATTN_DEVSTATUS_BAD_BLOCK", "ATTN_DEVSTATUS_BAD_SEQLEN",
 }
 
 

@@ -16,6 +16,9 @@ import torch
 library_path = os.path.join(os.path.dirname(os.path.abspath(__file__)), "_lib", "libattn_b200.so")
 
 ATTN_OK = 0
+ATTN_DEVSTATUS_TIMEOUT = 0x1
+ATTN_DEVSTATUS_BAD_BLOCK = 0x2
+ATTN_DEVSTATUS_BAD_SEQLEN = 0x4
 _lib = None
 
 
@@ -51,6 +54,15 @@ def library() -> ctypes.CDLL:
         lib.paged_attn_decode_fp8.restype = c_int
         lib.paged_attn_decode_noalloc.argtypes = lib.paged_attn_decode.argtypes
         lib.paged_attn_decode_noalloc.restype = c_int
+        lib.paged_attn_decode_checked.argtypes = [vp, vp, vp, vp, vp, c_int, c_int, c_int, c_int, c_int, c_int,
+                                                  c_int, c_int, vp, vp]
+        lib.paged_attn_decode_checked.restype = c_int
+        lib.paged_attn_decode_fp8_checked.argtypes = [vp, vp, vp, vp, vp, c_int, c_int, c_int, c_int, c_int, c_int,
+                                                      c_int, c_int, c_float, c_float, vp, vp]
+        lib.paged_attn_decode_fp8_checked.restype = c_int
+        lib.paged_attn_prefill_checked.argtypes = [vp, vp, vp, vp, vp, vp, c_int, c_int, c_int, c_int, c_int, c_int,
+                                                   c_int, c_int, c_int, c_int, c_float, vp, vp, vp]
+        lib.paged_attn_prefill_checked.restype = c_int
         lib.attn_check_support.argtypes = [c_int]
         lib.attn_check_support.restype = c_int
         lib.attn_status_string.argtypes = [c_int]
@@ -134,6 +146,42 @@ def paged_attn_decode_fp8(q, k_cache, v_cache, block_table, seq_lens, B, Hq, Hkv
                                          int(num_splits), float(k_scale), float(v_scale), _ptr(o), _stream(stream))
     if rc != ATTN_OK:
         raise AttnError(rc, "paged_attn_decode_fp8")
+
+
+def paged_attn_decode_checked(q, k_cache, v_cache, block_table, seq_lens, B, Hq, Hkv, d, block_size, max_blocks,
+                              num_blocks, num_splits, o, stream=None) -> None:
+    """paged_attn_decode for a pool of num_blocks blocks: table entries
+    outside it are masked and flagged (see attn.h)."""
+    rc = library().paged_attn_decode_checked(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_table),
+                                             _ptr(seq_lens), int(B), int(Hq), int(Hkv), int(d), int(block_size),
+                                             int(max_blocks), int(num_blocks), int(num_splits), _ptr(o),
+                                             _stream(stream))
+    if rc != ATTN_OK:
+        raise AttnError(rc, "paged_attn_decode_checked")
+
+
+def paged_attn_decode_fp8_checked(q, k_cache, v_cache, block_table, seq_lens, B, Hq, Hkv, d, block_size, max_blocks,
+                                  num_blocks, num_splits, k_scale, v_scale, o, stream=None) -> None:
+    """paged_attn_decode_fp8 for a pool of num_blocks blocks (see attn.h)."""
+    rc = library().paged_attn_decode_fp8_checked(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_table),
+                                                 _ptr(seq_lens), int(B), int(Hq), int(Hkv), int(d), int(block_size),
+                                                 int(max_blocks), int(num_blocks), int(num_splits), float(k_scale),
+                                                 float(v_scale), _ptr(o), _stream(stream))
+    if rc != ATTN_OK:
+        raise AttnError(rc, "paged_attn_decode_fp8_checked")
+
+
+def paged_attn_prefill_checked(q, k_cache, v_cache, block_table, seq_lens, cu_seqlens_q, B, Hq, Hkv, d, block_size,
+                               max_blocks, num_blocks, max_seqlen_q, total_q, causal, scale, o, lse,
+                               stream=None) -> None:
+    """paged_attn_prefill for a pool of num_blocks blocks (see attn.h)."""
+    rc = library().paged_attn_prefill_checked(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_table),
+                                              _ptr(seq_lens), _ptr(cu_seqlens_q), int(B), int(Hq), int(Hkv), int(d),
+                                              int(block_size), int(max_blocks), int(num_blocks), int(max_seqlen_q),
+                                              int(total_q), int(bool(causal)), float(scale), _ptr(o), _ptr(lse),
+                                              _stream(stream))
+    if rc != ATTN_OK:
+        raise AttnError(rc, "paged_attn_prefill_checked")
 
 
 def paged_attn_decode_noalloc(q, k_cache, v_cache, block_table, seq_lens, B, Hq, Hkv, d, block_size,

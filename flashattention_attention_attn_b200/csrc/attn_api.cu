@@ -151,12 +151,13 @@ int make_map_bthd(CUtensorMap* map, const void* base, int B, int rows, int H, in
   return r == CUDA_SUCCESS ? ATTN_OK : ATTN_ERR_CUDA;
 }
 
-// 2-D bf16 map over a paged pool seen as [tokens, Hkv * D]: box (64, 16).
-// The pool size is not part of the call, so the token extent is the largest
-// the coordinates can address; only block ids read from the table are used.
-int make_map_pool(CUtensorMap* map, const void* base, int Hkv, int D) {
-  constexpr cuuint64_t kTokens = (1ull << 31) - 16;
-  cuuint64_t dims[2] = {cuuint64_t(Hkv) * D, kTokens};
+// 2-D bf16 map over a paged pool of num_blocks 16-token blocks seen as
+// [tokens, Hkv * D]: box (64, 16).  When the caller does not give the pool
+// size, num_blocks is kMaxPoolBlocks (the largest count int32 token
+// coordinates address); the kernels load only ids below num_blocks.
+int make_map_pool(CUtensorMap* map, const void* base, int Hkv, int D, int num_blocks) {
+  const cuuint64_t tokens = cuuint64_t(num_blocks) * decode::kBlock;
+  cuuint64_t dims[2] = {cuuint64_t(Hkv) * D, tokens};
   cuuint64_t strides[1] = {cuuint64_t(Hkv) * D * 2};
   cuuint32_t box[2] = {64, 16};
   cuuint32_t estr[2] = {1, 1};
@@ -172,10 +173,10 @@ int make_map_pool(CUtensorMap* map, const void* base, int Hkv, int D) {
 // (row, 16 tokens, rows_per_group) lands in shared memory as
 // [row of the group][token][128 bytes] -- one copy per tensor and block.
 int make_map_pool_group(CUtensorMap* map, const void* base, CUtensorMapDataType dt, int elem_bytes,
-                        int rows_per_token, int rows_per_group) {
-  constexpr cuuint64_t kTokens = (1ull << 31) - 16;
+                        int rows_per_token, int rows_per_group, int num_blocks) {
+  const cuuint64_t tokens = cuuint64_t(num_blocks) * decode::kBlock;
   const cuuint32_t row_elems = 128 / elem_bytes;
-  cuuint64_t dims[3] = {row_elems, kTokens, cuuint64_t(rows_per_token)};
+  cuuint64_t dims[3] = {row_elems, tokens, cuuint64_t(rows_per_token)};
   cuuint64_t strides[2] = {cuuint64_t(rows_per_token) * 128, 128};
   cuuint32_t box[3] = {row_elems, 16, cuuint32_t(rows_per_group)};
   cuuint32_t estr[3] = {1, 1, 1};
@@ -185,12 +186,13 @@ int make_map_pool_group(CUtensorMap* map, const void* base, CUtensorMapDataType 
   return r == CUDA_SUCCESS ? ATTN_OK : ATTN_ERR_CUDA;
 }
 
-int make_map_decode_bf16(CUtensorMap* map, const void* base, int Hkv, int D) {
-  return make_map_pool_group(map, base, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, Hkv * D / 64, decode::kKH * D / 64);
+int make_map_decode_bf16(CUtensorMap* map, const void* base, int Hkv, int D, int num_blocks) {
+  return make_map_pool_group(map, base, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, Hkv * D / 64, decode::kKH * D / 64,
+                             num_blocks);
 }
 
-int make_map_decode_fp8(CUtensorMap* map, const void* base, int Hkv) {
-  return make_map_pool_group(map, base, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, Hkv, decode::kKH);
+int make_map_decode_fp8(CUtensorMap* map, const void* base, int Hkv, int num_blocks) {
+  return make_map_pool_group(map, base, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, Hkv, decode::kKH, num_blocks);
 }
 
 int launch_status() {
@@ -298,9 +300,10 @@ int launch_prefill_varlen(const void* q, const void* k, const void* v, void* o, 
 template <int D>
 int launch_prefill_paged(const void* q, const void* kc, const void* vc, const int32_t* table, const int32_t* lens,
                          const int32_t* cu_q, void* o, float* lse, int B, int max_q, int total_q, int Hq, int Hkv,
-                         int max_blocks, int causal, float scale, cudaStream_t stream) {
+                         int max_blocks, int num_blocks, int causal, float scale, cudaStream_t stream) {
   CUtensorMap mq, mk, mv;
-  if (make_map_bthd(&mq, q, 1, total_q, Hq, D) || make_map_pool(&mk, kc, Hkv, D) || make_map_pool(&mv, vc, Hkv, D))
+  if (make_map_bthd(&mq, q, 1, total_q, Hq, D) || make_map_pool(&mk, kc, Hkv, D, num_blocks) ||
+      make_map_pool(&mv, vc, Hkv, D, num_blocks))
     return ATTN_ERR_CUDA;
   prefill::Params p;
   std::memset(&p, 0, sizeof(p));
@@ -310,6 +313,7 @@ int launch_prefill_paged(const void* q, const void* kc, const void* vc, const in
   p.block_table = table;
   p.seq_lens = lens;
   p.max_blocks = max_blocks;
+  p.num_blocks = num_blocks;
   p.B = B;
   p.Hq = Hq;
   p.Hkv = Hkv;
@@ -364,7 +368,7 @@ int launch_combine_wpr(const decode::Params& p, const int32_t* lens, cudaStream_
   const float* po = p.part_o;
   const float* pl = p.part_lse;
   if (cudaLaunchKernelEx(&cfg, decode::lse_combine<D, WPR>, po, pl, lens, p.o, p.B, p.Hq, p.num_splits,
-                         p.chunk) != cudaSuccess) {
+                         p.chunk, p.max_blocks) != cudaSuccess) {
     cudaGetLastError();
     return ATTN_ERR_CUDA;
   }
@@ -384,10 +388,11 @@ int launch_combine(const decode::Params& p, const int32_t* lens, cudaStream_t st
 
 template <int D>
 int launch_decode(const void* q, const void* kc, const void* vc, const int32_t* table, const int32_t* lens, int B,
-                  int Hq, int Hkv, int max_blocks, int num_splits, void* o, cudaStream_t stream,
+                  int Hq, int Hkv, int max_blocks, int num_blocks, int num_splits, void* o, cudaStream_t stream,
                   const DeviceState* st) {
   CUtensorMap mk, mv;
-  if (make_map_decode_bf16(&mk, kc, Hkv, D) || make_map_decode_bf16(&mv, vc, Hkv, D)) return ATTN_ERR_CUDA;
+  if (make_map_decode_bf16(&mk, kc, Hkv, D, num_blocks) || make_map_decode_bf16(&mv, vc, Hkv, D, num_blocks))
+    return ATTN_ERR_CUDA;
   const int groups = (Hkv + decode::kKH - 1) / decode::kKH;
   if (num_splits <= 0) num_splits = auto_splits(B, groups, max_blocks, st->sms);
   if (num_splits > max_blocks) num_splits = max_blocks;
@@ -406,6 +411,7 @@ int launch_decode(const void* q, const void* kc, const void* vc, const int32_t* 
   p.Hq = Hq;
   p.Hkv = Hkv;
   p.max_blocks = max_blocks;
+  p.num_blocks = num_blocks;
   p.num_splits = num_splits;
   p.chunk = chunk;
   p.scale_log2 = (1.0f / std::sqrt(static_cast<float>(D))) * 1.4426950408889634f;
@@ -441,11 +447,12 @@ int launch_decode(const void* q, const void* kc, const void* vc, const int32_t* 
 
 // FP8 (e4m3) cache: the same split / combine structure, 128-dim heads.
 int launch_decode_fp8(const void* q, const void* kc, const void* vc, const int32_t* table, const int32_t* lens,
-                      int B, int Hq, int Hkv, int max_blocks, int num_splits, float k_scale, float v_scale, void* o,
-                      cudaStream_t stream, const DeviceState* st) {
+                      int B, int Hq, int Hkv, int max_blocks, int num_blocks, int num_splits, float k_scale,
+                      float v_scale, void* o, cudaStream_t stream, const DeviceState* st) {
   constexpr int D = decode::kFp8D;
   CUtensorMap mk, mv;
-  if (make_map_decode_fp8(&mk, kc, Hkv) || make_map_decode_fp8(&mv, vc, Hkv)) return ATTN_ERR_CUDA;
+  if (make_map_decode_fp8(&mk, kc, Hkv, num_blocks) || make_map_decode_fp8(&mv, vc, Hkv, num_blocks))
+    return ATTN_ERR_CUDA;
   const int groups = (Hkv + decode::kKH - 1) / decode::kKH;
   if (num_splits <= 0) num_splits = auto_splits(B, groups, max_blocks, st->sms, decode::kFp8CtasPerSm);
   if (num_splits > max_blocks) num_splits = max_blocks;
@@ -463,6 +470,7 @@ int launch_decode_fp8(const void* q, const void* kc, const void* vc, const int32
   p.Hq = Hq;
   p.Hkv = Hkv;
   p.max_blocks = max_blocks;
+  p.num_blocks = num_blocks;
   p.num_splits = num_splits;
   p.chunk = chunk;
   p.scale_log2 = (1.0f / std::sqrt(static_cast<float>(D))) * k_scale * 1.4426950408889634f;
@@ -499,31 +507,113 @@ int launch_decode_fp8(const void* q, const void* kc, const void* vc, const int32
 
 using namespace attn;
 
-extern "C" int paged_attn_decode_fp8(const void* q, const void* k_cache, const void* v_cache,
-                                     const int32_t* block_table, const int32_t* seq_lens, int B, int Hq, int Hkv,
-                                     int d, int block_size, int max_blocks, int num_splits, float k_scale,
-                                     float v_scale, void* o, attn_stream_t stream_) {
-  cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+namespace attn {
+namespace {
+
+// Host checks shared by the paged entry points.  num_blocks: the pool size
+// given by the caller (checked entry points) or kMaxPoolBlocks.
+int check_paged_common(int B, int Hq, int Hkv, int d, int block_size, int max_blocks, int num_blocks) {
   if (B < 0 || Hq <= 0 || Hkv <= 0 || d <= 0 || block_size <= 0) return ATTN_ERR_INVALID_ARG;
   if (Hq % Hkv != 0) return ATTN_ERR_INVALID_ARG;
+  if (B == 0) return ATTN_OK;
+  if (max_blocks <= 0 || num_blocks <= 0) return ATTN_ERR_INVALID_ARG;
+  if (max_blocks > kMaxPoolBlocks || num_blocks > kMaxPoolBlocks) return ATTN_ERR_UNSUPPORTED;
+  if (block_size != decode::kBlock) return ATTN_ERR_UNSUPPORTED;
+  return ATTN_OK;
+}
+
+int decode_fp8_entry(const void* q, const void* k_cache, const void* v_cache, const int32_t* block_table,
+                     const int32_t* seq_lens, int B, int Hq, int Hkv, int d, int block_size, int max_blocks,
+                     int num_blocks, int num_splits, float k_scale, float v_scale, void* o, cudaStream_t stream) {
+  if (B < 0 || Hq <= 0 || Hkv <= 0 || d <= 0 || block_size <= 0) return ATTN_ERR_INVALID_ARG;
   if (!(k_scale > 0.f) || !std::isfinite(k_scale) || !(v_scale > 0.f) || !std::isfinite(v_scale))
     return ATTN_ERR_INVALID_ARG;
-  if (B == 0) return ATTN_OK;
-  if (max_blocks <= 0) return ATTN_ERR_INVALID_ARG;
+  int rc = check_paged_common(B, Hq, Hkv, d, block_size, max_blocks, num_blocks);
+  if (rc != ATTN_OK || B == 0) return rc;
   if (q == nullptr || k_cache == nullptr || v_cache == nullptr || block_table == nullptr || seq_lens == nullptr ||
       o == nullptr)
     return ATTN_ERR_INVALID_ARG;
   if (d != decode::kFp8D) return ATTN_ERR_UNSUPPORTED;
-  if (block_size != decode::kBlock) return ATTN_ERR_UNSUPPORTED;
   if (Hq / Hkv > 8) return ATTN_ERR_UNSUPPORTED;
   if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(o)) return ATTN_ERR_UNSUPPORTED;
   if ((reinterpret_cast<uintptr_t>(block_table) & 3u) || (reinterpret_cast<uintptr_t>(seq_lens) & 3u))
     return ATTN_ERR_UNSUPPORTED;
   DeviceState* st = nullptr;
-  int rc = current_device_state(&st);
+  rc = current_device_state(&st);
   if (rc != ATTN_OK) return rc;
-  return launch_decode_fp8(q, k_cache, v_cache, block_table, seq_lens, B, Hq, Hkv, max_blocks, num_splits, k_scale,
-                           v_scale, o, stream, st);
+  return launch_decode_fp8(q, k_cache, v_cache, block_table, seq_lens, B, Hq, Hkv, max_blocks, num_blocks,
+                           num_splits, k_scale, v_scale, o, stream, st);
+}
+
+int decode_entry(const void* q, const void* k_cache, const void* v_cache, const int32_t* block_table,
+                 const int32_t* seq_lens, int B, int Hq, int Hkv, int d, int block_size, int max_blocks,
+                 int num_blocks, int num_splits, void* o, cudaStream_t stream) {
+  int rc = check_paged_common(B, Hq, Hkv, d, block_size, max_blocks, num_blocks);
+  if (rc != ATTN_OK || B == 0) return rc;
+  if (q == nullptr || k_cache == nullptr || v_cache == nullptr || block_table == nullptr || seq_lens == nullptr ||
+      o == nullptr)
+    return ATTN_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return ATTN_ERR_UNSUPPORTED;
+  if (Hq / Hkv > 8) return ATTN_ERR_UNSUPPORTED;
+  if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(o)) return ATTN_ERR_UNSUPPORTED;
+  if ((reinterpret_cast<uintptr_t>(block_table) & 3u) || (reinterpret_cast<uintptr_t>(seq_lens) & 3u))
+    return ATTN_ERR_UNSUPPORTED;
+  DeviceState* st = nullptr;
+  rc = current_device_state(&st);
+  if (rc != ATTN_OK) return rc;
+  if (d == 64)
+    return launch_decode<64>(q, k_cache, v_cache, block_table, seq_lens, B, Hq, Hkv, max_blocks, num_blocks,
+                             num_splits, o, stream, st);
+  return launch_decode<128>(q, k_cache, v_cache, block_table, seq_lens, B, Hq, Hkv, max_blocks, num_blocks,
+                            num_splits, o, stream, st);
+}
+
+int prefill_paged_entry(const void* q, const void* k_cache, const void* v_cache, const int32_t* block_table,
+                        const int32_t* seq_lens, const int32_t* cu_seqlens_q, int B, int Hq, int Hkv, int d,
+                        int block_size, int max_blocks, int num_blocks, int max_seqlen_q, int total_q, int causal,
+                        float scale, void* o, float* lse, cudaStream_t stream) {
+  if (max_seqlen_q < 0 || total_q < 0) return ATTN_ERR_INVALID_ARG;
+  if (!(scale > 0.f) || !std::isfinite(scale)) return ATTN_ERR_INVALID_ARG;
+  int rc = check_paged_common(B, Hq, Hkv, d, block_size, max_blocks, num_blocks);
+  if (rc != ATTN_OK) return rc;
+  if (B == 0 || total_q == 0 || max_seqlen_q == 0) return ATTN_OK;
+  if (q == nullptr || k_cache == nullptr || v_cache == nullptr || block_table == nullptr || seq_lens == nullptr ||
+      cu_seqlens_q == nullptr || o == nullptr)
+    return ATTN_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return ATTN_ERR_UNSUPPORTED;
+  if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(o)) return ATTN_ERR_UNSUPPORTED;
+  if ((lse != nullptr && (reinterpret_cast<uintptr_t>(lse) & 3u)) ||
+      (reinterpret_cast<uintptr_t>(block_table) & 3u) || (reinterpret_cast<uintptr_t>(seq_lens) & 3u) ||
+      (reinterpret_cast<uintptr_t>(cu_seqlens_q) & 3u))
+    return ATTN_ERR_UNSUPPORTED;
+  DeviceState* st = nullptr;
+  rc = current_device_state(&st);
+  if (rc != ATTN_OK) return rc;
+  if (d == 64)
+    return launch_prefill_paged<64>(q, k_cache, v_cache, block_table, seq_lens, cu_seqlens_q, o, lse, B,
+                                    max_seqlen_q, total_q, Hq, Hkv, max_blocks, num_blocks, causal, scale, stream);
+  return launch_prefill_paged<128>(q, k_cache, v_cache, block_table, seq_lens, cu_seqlens_q, o, lse, B,
+                                   max_seqlen_q, total_q, Hq, Hkv, max_blocks, num_blocks, causal, scale, stream);
+}
+
+}  // namespace
+}  // namespace attn
+
+extern "C" int paged_attn_decode_fp8(const void* q, const void* k_cache, const void* v_cache,
+                                     const int32_t* block_table, const int32_t* seq_lens, int B, int Hq, int Hkv,
+                                     int d, int block_size, int max_blocks, int num_splits, float k_scale,
+                                     float v_scale, void* o, attn_stream_t stream) {
+  return decode_fp8_entry(q, k_cache, v_cache, block_table, seq_lens, B, Hq, Hkv, d, block_size, max_blocks,
+                          kMaxPoolBlocks, num_splits, k_scale, v_scale, o, reinterpret_cast<cudaStream_t>(stream));
+}
+
+extern "C" int paged_attn_decode_fp8_checked(const void* q, const void* k_cache, const void* v_cache,
+                                             const int32_t* block_table, const int32_t* seq_lens, int B, int Hq,
+                                             int Hkv, int d, int block_size, int max_blocks, int num_blocks,
+                                             int num_splits, float k_scale, float v_scale, void* o,
+                                             attn_stream_t stream) {
+  return decode_fp8_entry(q, k_cache, v_cache, block_table, seq_lens, B, Hq, Hkv, d, block_size, max_blocks,
+                          num_blocks, num_splits, k_scale, v_scale, o, reinterpret_cast<cudaStream_t>(stream));
 }
 
 extern "C" int attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq, int Hkv,
@@ -586,59 +676,35 @@ extern "C" int attn_fwd_varlen(const void* q, const void* k, const void* v, void
 extern "C" int paged_attn_prefill(const void* q, const void* k_cache, const void* v_cache,
                                   const int32_t* block_table, const int32_t* seq_lens, const int32_t* cu_seqlens_q,
                                   int B, int Hq, int Hkv, int d, int block_size, int max_blocks, int max_seqlen_q,
-                                  int total_q, int causal, float scale, void* o, float* lse, attn_stream_t stream_) {
-  cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
-  if (B < 0 || Hq <= 0 || Hkv <= 0 || d <= 0 || block_size <= 0 || max_seqlen_q < 0 || total_q < 0)
-    return ATTN_ERR_INVALID_ARG;
-  if (Hq % Hkv != 0) return ATTN_ERR_INVALID_ARG;
-  if (!(scale > 0.f) || !std::isfinite(scale)) return ATTN_ERR_INVALID_ARG;
-  if (B == 0 || total_q == 0 || max_seqlen_q == 0) return ATTN_OK;
-  if (max_blocks <= 0) return ATTN_ERR_INVALID_ARG;
-  if (q == nullptr || k_cache == nullptr || v_cache == nullptr || block_table == nullptr || seq_lens == nullptr ||
-      cu_seqlens_q == nullptr || o == nullptr)
-    return ATTN_ERR_INVALID_ARG;
-  if (d != 64 && d != 128) return ATTN_ERR_UNSUPPORTED;
-  if (block_size != decode::kBlock) return ATTN_ERR_UNSUPPORTED;
-  if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(o)) return ATTN_ERR_UNSUPPORTED;
-  if ((lse != nullptr && (reinterpret_cast<uintptr_t>(lse) & 3u)) ||
-      (reinterpret_cast<uintptr_t>(block_table) & 3u) || (reinterpret_cast<uintptr_t>(seq_lens) & 3u) ||
-      (reinterpret_cast<uintptr_t>(cu_seqlens_q) & 3u))
-    return ATTN_ERR_UNSUPPORTED;
-  DeviceState* st = nullptr;
-  int rc = current_device_state(&st);
-  if (rc != ATTN_OK) return rc;
-  if (d == 64)
-    return launch_prefill_paged<64>(q, k_cache, v_cache, block_table, seq_lens, cu_seqlens_q, o, lse, B,
-                                    max_seqlen_q, total_q, Hq, Hkv, max_blocks, causal, scale, stream);
-  return launch_prefill_paged<128>(q, k_cache, v_cache, block_table, seq_lens, cu_seqlens_q, o, lse, B,
-                                   max_seqlen_q, total_q, Hq, Hkv, max_blocks, causal, scale, stream);
+                                  int total_q, int causal, float scale, void* o, float* lse, attn_stream_t stream) {
+  return prefill_paged_entry(q, k_cache, v_cache, block_table, seq_lens, cu_seqlens_q, B, Hq, Hkv, d, block_size,
+                             max_blocks, kMaxPoolBlocks, max_seqlen_q, total_q, causal, scale, o, lse,
+                             reinterpret_cast<cudaStream_t>(stream));
+}
+
+extern "C" int paged_attn_prefill_checked(const void* q, const void* k_cache, const void* v_cache,
+                                          const int32_t* block_table, const int32_t* seq_lens,
+                                          const int32_t* cu_seqlens_q, int B, int Hq, int Hkv, int d, int block_size,
+                                          int max_blocks, int num_blocks, int max_seqlen_q, int total_q, int causal,
+                                          float scale, void* o, float* lse, attn_stream_t stream) {
+  return prefill_paged_entry(q, k_cache, v_cache, block_table, seq_lens, cu_seqlens_q, B, Hq, Hkv, d, block_size,
+                             max_blocks, num_blocks, max_seqlen_q, total_q, causal, scale, o, lse,
+                             reinterpret_cast<cudaStream_t>(stream));
 }
 
 extern "C" int paged_attn_decode(const void* q, const void* k_cache, const void* v_cache,
                                  const int32_t* block_table, const int32_t* seq_lens, int B, int Hq, int Hkv, int d,
-                                 int block_size, int max_blocks, int num_splits, void* o, attn_stream_t stream_) {
-  cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
-  if (B < 0 || Hq <= 0 || Hkv <= 0 || d <= 0 || block_size <= 0) return ATTN_ERR_INVALID_ARG;
-  if (Hq % Hkv != 0) return ATTN_ERR_INVALID_ARG;
-  if (B == 0) return ATTN_OK;
-  if (max_blocks <= 0) return ATTN_ERR_INVALID_ARG;
-  if (q == nullptr || k_cache == nullptr || v_cache == nullptr || block_table == nullptr || seq_lens == nullptr ||
-      o == nullptr)
-    return ATTN_ERR_INVALID_ARG;
-  if (d != 64 && d != 128) return ATTN_ERR_UNSUPPORTED;
-  if (block_size != decode::kBlock) return ATTN_ERR_UNSUPPORTED;
-  if (Hq / Hkv > 8) return ATTN_ERR_UNSUPPORTED;
-  if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(o)) return ATTN_ERR_UNSUPPORTED;
-  if ((reinterpret_cast<uintptr_t>(block_table) & 3u) || (reinterpret_cast<uintptr_t>(seq_lens) & 3u))
-    return ATTN_ERR_UNSUPPORTED;
-  DeviceState* st = nullptr;
-  int rc = current_device_state(&st);
-  if (rc != ATTN_OK) return rc;
-  if (d == 64)
-    return launch_decode<64>(q, k_cache, v_cache, block_table, seq_lens, B, Hq, Hkv, max_blocks, num_splits, o,
-                             stream, st);
-  return launch_decode<128>(q, k_cache, v_cache, block_table, seq_lens, B, Hq, Hkv, max_blocks, num_splits, o,
-                            stream, st);
+                                 int block_size, int max_blocks, int num_splits, void* o, attn_stream_t stream) {
+  return decode_entry(q, k_cache, v_cache, block_table, seq_lens, B, Hq, Hkv, d, block_size, max_blocks,
+                      kMaxPoolBlocks, num_splits, o, reinterpret_cast<cudaStream_t>(stream));
+}
+
+extern "C" int paged_attn_decode_checked(const void* q, const void* k_cache, const void* v_cache,
+                                         const int32_t* block_table, const int32_t* seq_lens, int B, int Hq, int Hkv,
+                                         int d, int block_size, int max_blocks, int num_blocks, int num_splits,
+                                         void* o, attn_stream_t stream) {
+  return decode_entry(q, k_cache, v_cache, block_table, seq_lens, B, Hq, Hkv, d, block_size, max_blocks,
+                      num_blocks, num_splits, o, reinterpret_cast<cudaStream_t>(stream));
 }
 
 extern "C" int attn_check_support(int device) {
@@ -767,7 +833,8 @@ int launch_decode_noalloc(const void* q, const void* kc, const void* vc, const i
   const size_t rows = static_cast<size_t>(num_splits) * B * Hq;
   if (num_splits > 1 && num_splits * row_bytes > ATTN_NOALLOC_SCRATCH_BYTES) return ATTN_ERR_UNSUPPORTED;
   CUtensorMap mk, mv;
-  if (make_map_decode_bf16(&mk, kc, Hkv, D) || make_map_decode_bf16(&mv, vc, Hkv, D)) return ATTN_ERR_CUDA;
+  if (make_map_decode_bf16(&mk, kc, Hkv, D, kMaxPoolBlocks) || make_map_decode_bf16(&mv, vc, Hkv, D, kMaxPoolBlocks))
+    return ATTN_ERR_CUDA;
 
   decode::Params p;
   p.q = static_cast<const __nv_bfloat16*>(q);
@@ -780,6 +847,7 @@ int launch_decode_noalloc(const void* q, const void* kc, const void* vc, const i
   p.Hq = Hq;
   p.Hkv = Hkv;
   p.max_blocks = max_blocks;
+  p.num_blocks = kMaxPoolBlocks;
   p.num_splits = num_splits;
   p.chunk = chunk;
   p.scale_log2 = (1.0f / std::sqrt(static_cast<float>(D))) * 1.4426950408889634f;
@@ -803,6 +871,7 @@ extern "C" int paged_attn_decode_noalloc(const void* q, const void* k_cache, con
   if (Hq % Hkv != 0) return ATTN_ERR_INVALID_ARG;
   if (B == 0) return ATTN_OK;
   if (max_blocks <= 0) return ATTN_ERR_INVALID_ARG;
+  if (max_blocks > kMaxPoolBlocks) return ATTN_ERR_UNSUPPORTED;
   if (q == nullptr || k_cache == nullptr || v_cache == nullptr || block_table == nullptr || seq_lens == nullptr ||
       o == nullptr)
     return ATTN_ERR_INVALID_ARG;

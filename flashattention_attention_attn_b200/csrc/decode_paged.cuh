@@ -25,6 +25,11 @@
 // Output: with one split the bf16 result is written directly; otherwise each
 // unit writes its normalised partial output (fp32) and its log-sum-exp, and
 // lse_combine merges the splits:  O = sum_i e^{lse_i - M} o_i / sum_i e^{lse_i - M}.
+//
+// Checks: a sequence length outside [0, max_blocks * 16] is clamped into it
+// (the table row holds no more blocks) and a block-table entry outside
+// [0, num_blocks) is never loaded: its 16 positions are left out of the
+// softmax.  Both set a bit of the device status word.
 #pragma once
 
 #include "sm100_ptx.cuh"
@@ -50,6 +55,7 @@ struct __align__(1024) Smem {
   __nv_bfloat16 k[kStages][kKH][C::kChunks][kBlock * 64];
   __nv_bfloat16 v[kStages][kKH][C::kChunks][kBlock * 64];
   uint64_t full[kStages], empty[kStages];
+  int bad[kStages];  // 1: the stage's block id lies outside the pool (nothing loaded)
   int abort_flag;
 };
 
@@ -66,10 +72,21 @@ struct Params {
   float* part_o;               // [num_splits, B, Hq, D]
   float* part_lse;             // [num_splits, B, Hq]
   int B, Hq, Hkv, max_blocks;
+  int num_blocks;              // pool size: block ids outside [0, num_blocks) are masked
   int num_splits, chunk;       // chunk = blocks per split
   float scale_log2;            // scale * log2(e) (FP8 path: scale * k_scale * log2(e))
   float v_scale = 1.0f;        // FP8 path: V = v_scale * v_cache
 };
+
+// Cached tokens of sequence b, clamped to what its table row can name; a
+// length outside that range sets kDevStatusBadSeqLen (by one thread, `report`).
+__device__ __forceinline__ int checked_len(const int32_t* seq_lens, int b, int max_blocks, bool report) {
+  const int L = seq_lens[b];
+  const int cap = max_blocks * kBlock;
+  if (L >= 0 && L <= cap) return L;
+  if (report) atomicOr(&g_devstatus, kDevStatusBadSeqLen);
+  return L < 0 ? 0 : cap;
+}
 
 // Byte address of token row t, 16-byte unit u of a 128-byte-swizzled chunk.
 __device__ __forceinline__ uint32_t sw128(uint32_t chunk_base, int t, int u) {
@@ -106,7 +123,7 @@ __global__ void __launch_bounds__((kKH + 1) * 32, 2)
   grid_dependency_wait();
   grid_launch_dependents();
 
-  const int L = p.seq_lens[b];
+  const int L = checked_len(p.seq_lens, b, p.max_blocks, threadIdx.x == 0 && split == 0 && hg == 0);
   const int nb = (L + kBlock - 1) / kBlock;
   const int blk0 = split * p.chunk;
   const int blk1 = min(nb, blk0 + p.chunk);
@@ -142,11 +159,19 @@ __global__ void __launch_bounds__((kKH + 1) * 32, 2)
         if (lane == 0) {
           ok = mbar_wait(&sm.empty[s], ((j / kStages) & 1) ^ 1, abort_flag);
           if (ok) {
-            // one copy per tensor: the 16 token rows of the group's kKH heads
-            // (heads past Hkv are zero-filled and still count as bytes)
-            mbar_arrive_expect_tx(&sm.full[s], 2 * kKH * C::kHeadBytes);
-            tma_load_3d(sm.k[s][0][0], &tmK, &sm.full[s], 0, phys * kBlock, hg * kKH * C::kChunks);
-            tma_load_3d(sm.v[s][0][0], &tmV, &sm.full[s], 0, phys * kBlock, hg * kKH * C::kChunks);
+            if (static_cast<unsigned>(phys) < static_cast<unsigned>(p.num_blocks)) {
+              // one copy per tensor: the 16 token rows of the group's kKH heads
+              // (heads past Hkv are zero-filled and still count as bytes)
+              sm.bad[s] = 0;
+              mbar_arrive_expect_tx(&sm.full[s], 2 * kKH * C::kHeadBytes);
+              tma_load_3d(sm.k[s][0][0], &tmK, &sm.full[s], 0, phys * kBlock, hg * kKH * C::kChunks);
+              tma_load_3d(sm.v[s][0][0], &tmV, &sm.full[s], 0, phys * kBlock, hg * kKH * C::kChunks);
+            } else {
+              // an id outside the pool: nothing is loaded, the consumers skip the block
+              sm.bad[s] = 1;
+              atomicOr(&g_devstatus, kDevStatusBadBlock);
+              mbar_arrive(&sm.full[s]);
+            }
             issued = j + 1;
           }
         }
@@ -199,6 +224,11 @@ __global__ void __launch_bounds__((kKH + 1) * 32, 2)
     const int s = j % kStages;
     ok = __all_sync(0xffffffffu, mbar_wait(&sm.full[s], (j / kStages) & 1, abort_flag));
     if (!ok) break;
+    if (sm.bad[s]) {  // a block outside the pool: its keys take no part (warp-uniform)
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&sm.empty[s]);
+      continue;
+    }
 
     // ---- S^T = K q^T over the 16 tokens of this block ----
     float sc[4] = {0.f, 0.f, 0.f, 0.f};
@@ -283,7 +313,8 @@ __global__ void __launch_bounds__((kKH + 1) * 32, 2)
     l1 += __shfl_xor_sync(0xffffffffu, l1, off);
   }
   if (!ok) return;
-  const float inv0 = 1.0f / l0, inv1 = 1.0f / l1;
+  // l = 0 only when every block of the range lay outside the pool: O = 0, LSE = -inf
+  const float inv0 = l0 > 0.f ? 1.0f / l0 : 0.f, inv1 = l1 > 0.f ? 1.0f / l1 : 0.f;
   const int g0 = 2 * quad, g1 = 2 * quad + 1;
   const size_t head0 = static_cast<size_t>(b) * p.Hq + hk * G;  // first query head of this kv head
   if (p.num_splits == 1) {
@@ -341,7 +372,7 @@ template <int D, int WPR>
 __global__ void __launch_bounds__(CombineShape<WPR>::kWarps * 32)
     lse_combine(const float* __restrict__ part_o, const float* __restrict__ part_lse,
                 const int32_t* __restrict__ seq_lens, __nv_bfloat16* __restrict__ o, int B, int Hq,
-                int num_splits, int chunk) {
+                int num_splits, int chunk, int max_blocks) {
   using Shape = CombineShape<WPR>;
   constexpr int kPer = D / 32;
   constexpr int kUnroll = (WPR == 1) ? 8 : 4;  // rows in flight per lane: one round for up to 8 splits
@@ -359,7 +390,7 @@ __global__ void __launch_bounds__(CombineShape<WPR>::kWarps * 32)
   grid_launch_dependents();
   int nsp = 0;
   if (live) {
-    const int L = seq_lens[row_id / Hq];
+    const int L = checked_len(seq_lens, row_id / Hq, max_blocks, false);  // the split kernel reports
     nsp = min(num_splits, (((L + kBlock - 1) / kBlock) + chunk - 1) / chunk);  // splits holding data
   }
   const size_t stride = static_cast<size_t>(B) * Hq;  // rows between splits
@@ -388,6 +419,7 @@ __global__ void __launch_bounds__(CombineShape<WPR>::kWarps * 32)
     float mx = m;
 #pragma unroll
     for (int u = 0; u < kUnroll; ++u) mx = fmaxf(mx, lv[u]);
+    if (mx == -INFINITY) continue;  // no keys in these splits so far (all outside the pool)
     const float sc = ex2_approx(m - mx);  // m = -inf on the first round: 0
     wsum *= sc;
 #pragma unroll
@@ -404,7 +436,7 @@ __global__ void __launch_bounds__(CombineShape<WPR>::kWarps * 32)
   if constexpr (WPR == 1) {
     if (!live) return;
     __nv_bfloat16* out = o + static_cast<size_t>(row_id) * D + lane * kPer;
-    const float inv = (nsp > 0) ? 1.0f / wsum : 0.f;  // empty sequence: O = 0
+    const float inv = (wsum > 0.f) ? 1.0f / wsum : 0.f;  // no key at all: O = 0
 #pragma unroll
     for (int e = 0; e < kPer; ++e) out[e] = __float2bfloat16_rn(acc[e] * inv);
     return;
@@ -418,16 +450,16 @@ __global__ void __launch_bounds__(CombineShape<WPR>::kWarps * 32)
     __syncthreads();
     if (!live || sub != 0) return;
     __nv_bfloat16* out = o + static_cast<size_t>(row_id) * D + lane * kPer;
-    if (nsp == 0) {  // empty sequence: O = 0
-#pragma unroll
-      for (int e = 0; e < kPer; ++e) out[e] = __float2bfloat16_rn(0.f);
-      return;
-    }
     // the first warp of the row merges its WPR warps
     const int w0 = local_row * WPR;
     float M = -INFINITY;
 #pragma unroll
     for (int w = 0; w < WPR; ++w) M = fmaxf(M, s_m[w0 + w]);
+    if (M == -INFINITY) {  // empty sequence, or no key inside the pool: O = 0
+#pragma unroll
+      for (int e = 0; e < kPer; ++e) out[e] = __float2bfloat16_rn(0.f);
+      return;
+    }
     float ws = 0.f;
     float tot[kPer];
 #pragma unroll

@@ -22,7 +22,8 @@
 // over the two tokens for column 2j and one for column 2j+1, which become
 // the A-fragment rows j and j + 8: each 16-row output tile holds its 16
 // columns in the order (0, 2, .., 14, 1, 3, .., 15).  v_scale is applied
-// once at the end.
+// once at the end.  Sequence lengths and block ids are checked as in
+// paged_decode_split.
 #pragma once
 
 #include "decode_paged.cuh"
@@ -43,6 +44,7 @@ struct __align__(1024) SmemFp8 {
   uint8_t k[kFp8Stages][kKH][kFp8HeadBytes];
   uint8_t v[kFp8Stages][kKH][kFp8HeadBytes];
   uint64_t full[kFp8Stages], empty[kFp8Stages];
+  int bad[kFp8Stages];  // 1: the stage's block id lies outside the pool (nothing loaded)
   int abort_flag;
 };
 
@@ -74,7 +76,7 @@ __global__ void __launch_bounds__((kKH + 1) * 32, kFp8CtasPerSm)
   grid_dependency_wait();
   grid_launch_dependents();
 
-  const int L = p.seq_lens[b];
+  const int L = checked_len(p.seq_lens, b, p.max_blocks, threadIdx.x == 0 && split == 0 && hg == 0);
   const int nb = (L + kBlock - 1) / kBlock;
   const int blk0 = split * p.chunk;
   const int blk1 = min(nb, blk0 + p.chunk);
@@ -106,11 +108,19 @@ __global__ void __launch_bounds__((kKH + 1) * 32, kFp8CtasPerSm)
         if (lane == 0) {
           ok = mbar_wait(&sm.empty[s], ((j / kFp8Stages) & 1) ^ 1, abort_flag);
           if (ok) {
-            // one copy per tensor: the 16 token rows of the group's kKH heads
-            // (heads past Hkv are zero-filled and still count as bytes)
-            mbar_arrive_expect_tx(&sm.full[s], 2 * kKH * kFp8HeadBytes);
-            tma_load_3d(sm.k[s][0], &tmK, &sm.full[s], 0, phys * kBlock, hg * kKH);
-            tma_load_3d(sm.v[s][0], &tmV, &sm.full[s], 0, phys * kBlock, hg * kKH);
+            if (static_cast<unsigned>(phys) < static_cast<unsigned>(p.num_blocks)) {
+              // one copy per tensor: the 16 token rows of the group's kKH heads
+              // (heads past Hkv are zero-filled and still count as bytes)
+              sm.bad[s] = 0;
+              mbar_arrive_expect_tx(&sm.full[s], 2 * kKH * kFp8HeadBytes);
+              tma_load_3d(sm.k[s][0], &tmK, &sm.full[s], 0, phys * kBlock, hg * kKH);
+              tma_load_3d(sm.v[s][0], &tmV, &sm.full[s], 0, phys * kBlock, hg * kKH);
+            } else {
+              // an id outside the pool: nothing is loaded, the consumers skip the block
+              sm.bad[s] = 1;
+              atomicOr(&g_devstatus, kDevStatusBadBlock);
+              mbar_arrive(&sm.full[s]);
+            }
             issued = j + 1;
           }
         }
@@ -167,6 +177,11 @@ __global__ void __launch_bounds__((kKH + 1) * 32, kFp8CtasPerSm)
     const int s = j % kFp8Stages;
     ok = __all_sync(0xffffffffu, mbar_wait(&sm.full[s], (j / kFp8Stages) & 1, abort_flag));
     if (!ok) break;
+    if (sm.bad[s]) {  // a block outside the pool: its keys take no part (warp-uniform)
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&sm.empty[s]);
+      continue;
+    }
 
     // ---- S^T = K q^T (log2 domain) ----
     float sc[4] = {0.f, 0.f, 0.f, 0.f};
@@ -253,7 +268,8 @@ __global__ void __launch_bounds__((kKH + 1) * 32, kFp8CtasPerSm)
   }
   if (!ok) return;
   const int g0 = 2 * quad, g1 = 2 * quad + 1;
-  const float inv0 = p.v_scale / l0, inv1 = p.v_scale / l1;
+  // l = 0 only when every block of the range lay outside the pool: O = 0, LSE = -inf
+  const float inv0 = l0 > 0.f ? p.v_scale / l0 : 0.f, inv1 = l1 > 0.f ? p.v_scale / l1 : 0.f;
   const int j2 = 2 * g_row;  // this lane's even column within each 16-column tile
   const size_t head0 = static_cast<size_t>(b) * p.Hq + hk * G;
   if (p.num_splits == 1) {

@@ -91,6 +91,7 @@ struct Params {
   const int32_t* block_table;  // paged: [B, max_blocks] physical 16-token blocks
   const int32_t* seq_lens;     // paged: [B] cached tokens (keys) per sequence
   int max_blocks;
+  int num_blocks;              // paged: pool size; block ids outside [0, num_blocks) are masked
   int B, Hq, Hkv, T, S;   // dense: T, S; varlen: T = max query length
   int total_q;            // varlen: rows of the packed query tensor
   int causal;
@@ -114,7 +115,10 @@ __device__ __forceinline__ int kv_tiles_for(int r0, int T, int S, int causal) {
 // maps then cover [total, H, D] as batch 1 and each CTA takes its sequence's
 // row offset and length from cu_q.  kVarlen takes key rows from cu_k the
 // same way; kPaged reads every 128-key tile as eight 16-token blocks through
-// the block table (pool maps of [tokens, Hkv * D], box 64 x 16).
+// the block table (pool maps of [tokens, Hkv * D], box 64 x 16).  In kPaged
+// mode a sequence length is clamped to the table row's capacity and a block
+// id outside [0, num_blocks) is not loaded and its 16 keys are masked; both
+// set a bit of the device status word.
 template <int D, int MODE>
 __global__ void __launch_bounds__(kThreads, 1)
     prefill_fwd_sm100(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
@@ -208,7 +212,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     qoff = p.cu_q[b];
     T = p.cu_q[b + 1] - qoff;
     if constexpr (MODE == kPaged) {
+      // clamped to what the table row can name (flagged when outside)
       S = p.seq_lens[b];
+      if (S < 0 || S > p.max_blocks * 16) {
+        if (threadIdx.x == 0 && h == 0) atomicOr(&g_devstatus, kDevStatusBadSeqLen);
+        S = S < 0 ? 0 : p.max_blocks * 16;
+      }
     } else {
       koff = p.cu_k[b];
       S = p.cu_k[b + 1] - koff;
@@ -267,19 +276,34 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int j = pre; j < n_max; ++j) {
       const int s = j % C::kStages;
       const uint32_t ph = (j / C::kStages) & 1;
-      int nblk = kBlocks;    // 16-token blocks loaded into this tile
+      int nblk = kBlocks;    // 16-token blocks of this tile inside the sequence
       int valid = kBN;       // keys of this tile inside the sequence
       int my_id = 0;         // paged: physical block of this lane's copy
+      uint32_t bad = 0;      // paged: blocks of this tile whose id lies outside the pool
       if constexpr (MODE == kPaged) {
         valid = min(kBN, S - j * kBN);
         nblk = (valid + 15) / 16;
         const int mine = (lane < nblk) ? __ldg(p.block_table + static_cast<size_t>(b) * p.max_blocks +
                                                j * kBlocks + lane)
                                        : 0;
+        bad = __ballot_sync(0xffffffffu, lane < nblk && static_cast<unsigned>(mine) >=
+                                                            static_cast<unsigned>(p.num_blocks));
         my_id = __shfl_sync(0xffffffffu, mine, il);
+        if (bad && lane == 0) atomicOr(&g_devstatus, kDevStatusBadBlock);
       }
-      const bool my_copy = MODE == kPaged && cl < C::kChunks && il < nblk;
-      const uint32_t tile_bytes = static_cast<uint32_t>(nblk) * 16 * D * 2;
+      // blocks outside the pool are not loaded (the softmax masks their keys)
+      const bool my_copy = MODE == kPaged && cl < C::kChunks && il < nblk && !((bad >> il) & 1u);
+      const uint32_t tile_bytes = static_cast<uint32_t>(nblk - __popc(bad)) * 16 * D * 2;
+      // Rows of blocks outside the pool in a free V slot are cleared, so that
+      // a zero weight cannot meet a NaN left there.
+      auto clear_bad_rows = [&]() {
+        for (int i = lane; i < kBlocks * 16 * C::kChunks * 8; i += 32) {
+          const int unit = i & 7, c = (i >> 3) % C::kChunks, r = (i >> 3) / C::kChunks;
+          if ((bad >> (r / 16)) & 1u)
+            *reinterpret_cast<uint4*>(reinterpret_cast<uint8_t*>(sm.v[s][c]) + r * 128 + unit * 16) =
+                make_uint4(0u, 0u, 0u, 0u);
+        }
+      };
       bool ok = true;
       if (lane == 0) {
         ok = mbar_wait(&sm.kv_done[s], ph ^ 1, abort_flag);  // iteration j - kStages freed K's slot
@@ -322,10 +346,16 @@ __global__ void __launch_bounds__(kThreads, 1)
           *reinterpret_cast<uint4*>(reinterpret_cast<uint8_t*>(sm.v[s][c]) + r * 128 + unit * 16) =
               make_uint4(0u, 0u, 0u, 0u);
         }
+        if (bad) clear_bad_rows();
         fence_proxy_async_smem();  // the generic writes before the tensor core reads the tile
         __syncwarp();
         if (lane == 0) mbar_arrive(&sm.v_full[s]);
       } else {
+        if (MODE == kPaged && bad) {
+          clear_bad_rows();
+          fence_proxy_async_smem();  // before the arrive that hands the tile to the MMA
+          __syncwarp();
+        }
         if (lane == 0) {
           mbar_arrive_expect_tx(&sm.v_full[s], tile_bytes);
           if constexpr (MODE != kPaged) {
@@ -433,7 +463,17 @@ __global__ void __launch_bounds__(kThreads, 1)
     float m_used = -INFINITY;  // reference max, log2 domain
     float l = 0.f;             // running row sum relative to m_used
     bool ok = true;
+    // paged: lane i < 8 holds the table entry of block i of the next key
+    // tile (loaded one tile ahead); blocks outside the pool are masked
+    auto table_entry = [&](int jj) -> int {
+      const int nb = min(kBN / 16, (S - jj * kBN + 15) / 16);
+      return lane < nb ? __ldg(p.block_table + static_cast<size_t>(b) * p.max_blocks + jj * (kBN / 16) + lane)
+                       : 0;
+    };
+    int entry_next = (MODE == kPaged && nt > 0) ? table_entry(0) : 0;
     for (int j = 0; j < nt; ++j) {
+      const int entry = entry_next;
+      if (MODE == kPaged && j + 1 < nt) entry_next = table_entry(j + 1);
       ok = __all_sync(0xffffffffu, mbar_wait(&sm.s_full[t], j & 1, abort_flag));
       if (!ok) break;
       tc_fence_after();
@@ -449,6 +489,19 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int i = 0; i < kBN; ++i)
           if (i >= lim) s[i] = -INFINITY;
+      }
+      if constexpr (MODE == kPaged) {
+        const int nb = min(kBN / 16, (S - j * kBN + 15) / 16);
+        const uint32_t bad = __ballot_sync(0xffffffffu, lane < nb && static_cast<unsigned>(entry) >=
+                                                                         static_cast<unsigned>(p.num_blocks));
+        if (bad) {  // warp-uniform
+#pragma unroll
+          for (int g = 0; g < kBN / 16; ++g)
+            if ((bad >> g) & 1u) {
+#pragma unroll
+              for (int i = 0; i < 16; ++i) s[g * 16 + i] = -INFINITY;
+            }
+        }
       }
       // Row max with 3-input max: 8 independent chains of 16 scores each.
       float mx8[8];

@@ -16,6 +16,13 @@ namespace attn {
 // header), so this is its only definition.
 // ---------------------------------------------------------------------------
 __device__ int g_devstatus = 0;
+constexpr int kDevStatusTimeout = 0x1;    // a bounded wait gave up
+constexpr int kDevStatusBadBlock = 0x2;   // a block-table entry outside the pool (its keys were masked)
+constexpr int kDevStatusBadSeqLen = 0x4;  // a sequence length outside [0, max_blocks * block_size] (clamped)
+
+// Pool size assumed when the caller does not give one: the largest block
+// count whose token coordinates (16 per block) fit in int32.
+constexpr int kMaxPoolBlocks = (1 << 27) - 1;
 
 constexpr uint64_t kWaitLimitNs = 1000000000ull;  // 1 s: no legitimate wait is that long
 
@@ -74,7 +81,7 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
       if (*abort) return false;
       if (globaltimer_ns() - t0 > kWaitLimitNs) {
         *abort = 1;
-        atomicOr(&g_devstatus, 1);
+        atomicOr(&g_devstatus, kDevStatusTimeout);
         return false;
       }
     }
@@ -90,7 +97,7 @@ __device__ __forceinline__ bool mbar_wait_drain(uint64_t* bar, uint32_t parity) 
   for (uint32_t n = 1;; ++n) {
     if (mbar_try_wait(bar, parity)) return true;
     if ((n & 63u) == 0 && globaltimer_ns() - t0 > kWaitLimitNs) {
-      atomicOr(&g_devstatus, 1);
+      atomicOr(&g_devstatus, kDevStatusTimeout);
       return false;
     }
   }

@@ -65,6 +65,14 @@ typedef enum {
 
 /* Bits of the device status word (see attn_read_device_status). */
 #define ATTN_DEVSTATUS_TIMEOUT 0x1
+/* A paged call met a block-table entry outside the pool: the entry was not
+ * read through and its block_size positions were left out of the softmax
+ * (their keys masked).  Without a pool size (the unchecked entry points)
+ * only negative ids and ids of 2^27 - 1 or more are caught this way. */
+#define ATTN_DEVSTATUS_BAD_BLOCK 0x2
+/* A paged call met a seq_lens entry below 0 or above max_blocks * block_size
+ * (more positions than its table row names): it was clamped into that range. */
+#define ATTN_DEVSTATUS_BAD_SEQLEN 0x4
 
 /*
  * attn_fwd - dense prefill attention with grouped-query heads.
@@ -128,9 +136,16 @@ int attn_fwd_varlen(const void* q, const void* k, const void* v, void* o, float*
  *   v_cache      [num_blocks, block_size, Hkv, d]   bf16
  *   block_table  [B, max_blocks] int32: physical block of logical block j of
  *                sequence b.  Only entries j < ceil(seq_lens[b]/block_size)
- *                are read; they must be valid block ids of the pool.
+ *                are read; they must be valid block ids of the pool (the
+ *                pool's size is not an argument here: paged_attn_decode_checked
+ *                takes it and masks ids outside it; this entry point catches
+ *                only negative ids and ids >= 2^27 - 1, see
+ *                ATTN_DEVSTATUS_BAD_BLOCK).
  *   seq_lens     [B] int32: cached tokens of each sequence (0 allowed, which
- *                gives O = 0).  Must not exceed max_blocks * block_size.
+ *                gives O = 0).  A value below 0 or above
+ *                max_blocks * block_size is clamped into that range and sets
+ *                ATTN_DEVSTATUS_BAD_SEQLEN; no table entry past the row is
+ *                ever read.
  *   o            [B, Hq, d] bf16 (written)
  *
  *   The query of sequence b sits at position seq_lens[b]-1 and sees every
@@ -149,7 +164,7 @@ int attn_fwd_varlen(const void* q, const void* k, const void* v, void* o, float*
  *   cudaFreeAsync on `stream`).
  *
  *   Supported: d in {64, 128}; block_size == 16; 1 <= Hq/Hkv <= 8;
- *   sm_100 device; 16-byte aligned q, caches and o.
+ *   max_blocks < 2^27; sm_100 device; 16-byte aligned q, caches and o.
  *   Errors: as attn_fwd; ATTN_ERR_INVALID_ARG also for max_blocks <= 0 when
  *   B > 0.
  */
@@ -157,6 +172,32 @@ int paged_attn_decode(const void* q, const void* k_cache, const void* v_cache,
                       const int32_t* block_table, const int32_t* seq_lens,
                       int B, int Hq, int Hkv, int d, int block_size, int max_blocks,
                       int num_splits, void* o, attn_stream_t stream);
+
+/*
+ * paged_attn_decode_checked - paged_attn_decode for a pool of known size.
+ *
+ * The same translation through the block table ("De aandachtskernel moet
+ * dan elke positie via deze tabel vertalen", page "Snelle attention-kernels
+ * en operatorfusie versnellen AI-modellen", section "FlashAttention-type
+ * aandacht en gepagineerde aandacht"), with every id checked against the
+ * pool before it is used.
+ *
+ *   num_blocks  number of physical blocks in k_cache and v_cache (both
+ *               [num_blocks, block_size, Hkv, d]); 1 <= num_blocks < 2^27.
+ *   All other arguments, the result and the errors as paged_attn_decode;
+ *   ATTN_ERR_INVALID_ARG also for num_blocks <= 0 when B > 0.
+ *
+ *   An entry outside [0, num_blocks) among the entries a sequence reads
+ *   (j < ceil(seq_len / block_size)) is never dereferenced: its
+ *   block_size positions are left out of the softmax, as if masked, and
+ *   ATTN_DEVSTATUS_BAD_BLOCK is set.  A query whose every position is left
+ *   out gets O = 0.  The pool views the kernels load through end at
+ *   num_blocks as well, so no load reaches past the pool.
+ */
+int paged_attn_decode_checked(const void* q, const void* k_cache, const void* v_cache,
+                              const int32_t* block_table, const int32_t* seq_lens,
+                              int B, int Hq, int Hkv, int d, int block_size, int max_blocks,
+                              int num_blocks, int num_splits, void* o, attn_stream_t stream);
 
 /*
  * attn_check_support - initialisation-time compatibility check of `device`,
@@ -210,8 +251,10 @@ int attn_selftest_bounded_wait(attn_stream_t stream);
  *   causal != 0 it sees the keys at positions <= its own (bottom-right
  *   alignment of attn_fwd with T = T_b, S = seq_lens[b]); otherwise all
  *   seq_lens[b] keys.  Pool slots past the sequence end may hold anything.
- *   max_seqlen_q must be >= every T_b.
- *   Supported: d in {64, 128}; block_size == 16; Hq % Hkv == 0; sm_100.
+ *   max_seqlen_q must be >= every T_b.  seq_lens and block ids are checked
+ *   as in paged_attn_decode.
+ *   Supported: d in {64, 128}; block_size == 16; Hq % Hkv == 0;
+ *   max_blocks < 2^27; sm_100.
  *   Errors: as paged_attn_decode.
  */
 int paged_attn_prefill(const void* q, const void* k_cache, const void* v_cache,
@@ -219,6 +262,21 @@ int paged_attn_prefill(const void* q, const void* k_cache, const void* v_cache,
                        int B, int Hq, int Hkv, int d, int block_size, int max_blocks,
                        int max_seqlen_q, int total_q, int causal, float scale,
                        void* o, float* lse, attn_stream_t stream);
+
+/*
+ * paged_attn_prefill_checked - paged_attn_prefill for a pool of known size
+ * num_blocks (1 <= num_blocks < 2^27), with the block-id check of
+ * paged_attn_decode_checked: an entry outside [0, num_blocks) is never
+ * dereferenced, its positions are masked for every query row and
+ * ATTN_DEVSTATUS_BAD_BLOCK is set.  A row that sees no position gets O = 0
+ * and LSE = -inf.  Other arguments, results and errors as
+ * paged_attn_prefill.
+ */
+int paged_attn_prefill_checked(const void* q, const void* k_cache, const void* v_cache,
+                               const int32_t* block_table, const int32_t* seq_lens, const int32_t* cu_seqlens_q,
+                               int B, int Hq, int Hkv, int d, int block_size, int max_blocks, int num_blocks,
+                               int max_seqlen_q, int total_q, int causal, float scale,
+                               void* o, float* lse, attn_stream_t stream);
 
 /*
  * paged_attn_decode_fp8 - paged_attn_decode with the KV cache stored as FP8
@@ -238,6 +296,16 @@ int paged_attn_decode_fp8(const void* q, const void* k_cache, const void* v_cach
                           const int32_t* block_table, const int32_t* seq_lens,
                           int B, int Hq, int Hkv, int d, int block_size, int max_blocks,
                           int num_splits, float k_scale, float v_scale, void* o, attn_stream_t stream);
+
+/*
+ * paged_attn_decode_fp8_checked - paged_attn_decode_fp8 for a pool of known
+ * size num_blocks, with the block-id check of paged_attn_decode_checked.
+ */
+int paged_attn_decode_fp8_checked(const void* q, const void* k_cache, const void* v_cache,
+                                  const int32_t* block_table, const int32_t* seq_lens,
+                                  int B, int Hq, int Hkv, int d, int block_size, int max_blocks,
+                                  int num_blocks, int num_splits, float k_scale, float v_scale, void* o,
+                                  attn_stream_t stream);
 
 /*
  * paged_attn_decode_noalloc - paged_attn_decode for callers that must not
@@ -269,6 +337,7 @@ int paged_attn_decode_fp8(const void* q, const void* k_cache, const void* v_cach
  *   partial the merge reads is written earlier in the same call).  Calls that
  *   can overlap on the GPU (different streams without ordering between them)
  *   race on the scratch and give undefined results; serialise them.
+ *   seq_lens and block ids are checked as in paged_attn_decode.
  *   Errors: as paged_attn_decode, plus the limit above.
  */
 #define ATTN_NOALLOC_SCRATCH_BYTES (16u << 20)

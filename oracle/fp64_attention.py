@@ -33,6 +33,10 @@ Readings where the pages are silent (each listed in the design notes):
   * LSE is the natural log of the sum of exp of the *scaled* scores;
   * paged pool layout [num_blocks, block_size, Hkv, d]; block-table entries
     at or past ceil(seq_len / block_size) are never read;
+  * a seq_len beyond the table row's capacity (row length x block_size) is
+    clamped to it, a negative one to 0; when the pool size num_blocks is
+    known, a table entry outside [0, num_blocks) names no block of the pool
+    and its block_size positions are left out of the softmax (masked);
   * a decode query sits at position seq_len - 1 and sees all seq_len keys.
 
 Inputs are float64 numpy arrays (bf16 tensors are widened exactly by the
@@ -50,6 +54,7 @@ __all__ = [
     "softmax_rows",
     "attention",
     "attention_varlen",
+    "paged_positions",
     "gather_paged_kv",
     "paged_decode",
     "paged_prefill",
@@ -93,7 +98,7 @@ def softmax_rows(scores: np.ndarray, counts: np.ndarray):
     return P, m, l
 
 
-def attention(q, k, v, scale: float, causal: bool, rows=None):
+def attention(q, k, v, scale: float, causal: bool, rows=None, counts=None):
     """Softmax attention with grouped-query heads, fp64.
 
     q: [B, T, Hq, d]; k, v: [B, S, Hkv, d]  (float64)
@@ -102,6 +107,10 @@ def attention(q, k, v, scale: float, causal: bool, rows=None):
     ``rows``: optional sorted iterable of query rows to evaluate (the others
     are left at O = 0, LSE = -inf).  Used to sample outputs of workloads too
     large to evaluate whole.
+    ``counts``: optional [T] numbers of keys each row sees (keys
+    0..counts[i]-1), in place of the causal / non-causal rule.  Used where
+    some key positions of a paged cache are masked, so that the keys a row
+    sees are a prefix of the keys that remain.
     """
     q = np.asarray(q, dtype=np.float64)
     k = np.asarray(k, dtype=np.float64)
@@ -116,7 +125,10 @@ def attention(q, k, v, scale: float, causal: bool, rows=None):
     row_idx = np.arange(T) if rows is None else np.asarray(sorted(rows), dtype=np.int64)
     if row_idx.size == 0 or S == 0:
         return O, LSE
-    counts_all = np.array([visible_key_count(int(i), T, S, causal) for i in row_idx])
+    if counts is None:
+        counts_all = np.array([visible_key_count(int(i), T, S, causal) for i in row_idx])
+    else:
+        counts_all = np.asarray(counts, dtype=np.int64)[row_idx]
     for b in range(B):
         for h in range(Hq):
             hk = h // group  # grouped-query head map
@@ -157,47 +169,67 @@ def attention_varlen(q, k, v, cu_q, cu_k, scale: float, causal: bool):
     return O, LSE
 
 
-def gather_paged_kv(k_cache, v_cache, block_table_row, seq_len: int, block_size: int):
-    """Logical K/V of one sequence, read through its block-table row.
+def paged_positions(block_table_row, seq_len: int, block_size: int, num_blocks=None):
+    """The logical positions of one sequence that take part in attention.
 
     Position p lives in physical block block_table_row[p // block_size] at
     slot p % block_size ("De aandachtskernel moet dan elke positie via deze
-    tabel vertalen").  Only the first ceil(seq_len / block_size) entries of the
-    row are read.  Returns (K [L, Hkv, d], V [L, Hkv, d]) as views/copies of
-    the pool entries: the values are moved, never changed.
+    tabel vertalen").  Positions run from 0 to seq_len - 1, with seq_len
+    clamped to [0, len(row) * block_size] (the row cannot name more blocks).
+    With ``num_blocks`` (the pool size) given, positions whose block id lies
+    outside [0, num_blocks) are left out.  Only the table entries of
+    positions below the clamped seq_len are read.
+
+    Returns (pos, phys, slot, L): the kept positions (ascending), their
+    physical block and slot, and the clamped length L.
     """
-    L = int(seq_len)
+    row = np.asarray(block_table_row)
+    L = min(max(int(seq_len), 0), row.shape[0] * block_size)
     pos = np.arange(L)
-    logical_block = pos // block_size
-    phys = np.asarray(block_table_row)[logical_block].astype(np.int64)
+    phys = row[pos // block_size].astype(np.int64)
     slot = pos % block_size
+    if num_blocks is not None:
+        keep = (phys >= 0) & (phys < int(num_blocks))
+        pos, phys, slot = pos[keep], phys[keep], slot[keep]
+    return pos, phys, slot, L
+
+
+def gather_paged_kv(k_cache, v_cache, block_table_row, seq_len: int, block_size: int, num_blocks=None):
+    """Logical K/V of one sequence, read through its block-table row at the
+    positions ``paged_positions`` keeps.  Returns (K [n, Hkv, d],
+    V [n, Hkv, d]) as copies of the pool entries: the values are moved,
+    never changed.
+    """
+    _, phys, slot, _ = paged_positions(block_table_row, seq_len, block_size, num_blocks)
     return k_cache[phys, slot], v_cache[phys, slot]
 
 
-def paged_decode(q, k_cache, v_cache, block_table, seq_lens, block_size: int, scale: float):
+def paged_decode(q, k_cache, v_cache, block_table, seq_lens, block_size: int, scale: float, num_blocks=None):
     """Single-token decode against a paged KV cache, fp64.
 
-    q: [B, Hq, d]; k_cache, v_cache: [num_blocks, block_size, Hkv, d];
+    q: [B, Hq, d]; k_cache, v_cache: [pool, block_size, Hkv, d];
     block_table: [B, max_blocks] int; seq_lens: [B] int.
-    Each query sits at position seq_len - 1 and sees all seq_len cached keys.
-    Returns O [B, Hq, d], LSE [B, Hq].
+    Each query sits at position seq_len - 1 and sees all seq_len cached keys
+    (the positions ``paged_positions`` keeps; ``num_blocks``: the pool size,
+    when entries outside it are to be masked).  A query that sees no key
+    gets O = 0, LSE = -inf.  Returns O [B, Hq, d], LSE [B, Hq].
     """
     q = np.asarray(q, dtype=np.float64)
     B, Hq, d = q.shape
     O = np.zeros((B, Hq, d))
     LSE = np.full((B, Hq), -np.inf)
     for b in range(B):
-        L = int(seq_lens[b])
-        if L == 0:
+        Kb, Vb = gather_paged_kv(k_cache, v_cache, block_table[b], seq_lens[b], block_size, num_blocks)
+        if Kb.shape[0] == 0:
             continue
-        Kb, Vb = gather_paged_kv(k_cache, v_cache, block_table[b], L, block_size)
         ob, lb = attention(q[b][None, None], Kb[None], Vb[None], scale, causal=False)
         O[b] = ob[0, 0]
         LSE[b] = lb[0, :, 0]
     return O, LSE
 
 
-def paged_prefill(q, k_cache, v_cache, block_table, seq_lens, cu_q, block_size: int, scale: float, causal: bool):
+def paged_prefill(q, k_cache, v_cache, block_table, seq_lens, cu_q, block_size: int, scale: float, causal: bool,
+                  num_blocks=None):
     """Chunked prefill against a paged cache, fp64.
 
     q: [total_q, Hq, d] (the new tokens of every sequence, back to back,
@@ -205,8 +237,10 @@ def paged_prefill(q, k_cache, v_cache, block_table, seq_lens, cu_q, block_size: 
     sequence b, the new ones included as its last T_b tokens.  The logical
     K/V are gathered through the block table, then `attention` is applied
     with T = T_b and S = seq_lens[b] (bottom-right causal alignment: the new
-    token i sits at position S - T + i).  Returns O [total_q, Hq, d] and
-    LSE [Hq, total_q].
+    token i sits at position S - T + i and sees the positions up to its own).
+    Positions that ``paged_positions`` leaves out (``num_blocks`` given, an
+    entry outside the pool) are seen by no row; S is the clamped length.
+    Returns O [total_q, Hq, d] and LSE [Hq, total_q].
     """
     q = np.asarray(q, dtype=np.float64)
     total_q, Hq, d = q.shape
@@ -214,11 +248,15 @@ def paged_prefill(q, k_cache, v_cache, block_table, seq_lens, cu_q, block_size: 
     LSE = np.full((Hq, total_q), -np.inf)
     for b in range(len(cu_q) - 1):
         q0, q1 = int(cu_q[b]), int(cu_q[b + 1])
-        L = int(seq_lens[b])
         if q1 == q0:
             continue
-        Kb, Vb = gather_paged_kv(k_cache, v_cache, block_table[b], L, block_size)
-        ob, lb = attention(q[None, q0:q1], Kb[None], Vb[None], scale, causal)
+        pos, phys, slot, L = paged_positions(block_table[b], seq_lens[b], block_size, num_blocks)
+        Kb, Vb = k_cache[phys, slot], v_cache[phys, slot]
+        T = q1 - q0
+        # row i sees the kept positions p <= L - T + i (all of them if not causal)
+        limit = [L - T + i if causal else L - 1 for i in range(T)]
+        counts = np.searchsorted(pos, limit, side="right")
+        ob, lb = attention(q[None, q0:q1], Kb[None], Vb[None], scale, causal, counts=counts)
         O[q0:q1] = ob[0]
         LSE[:, q0:q1] = lb[0]
     return O, LSE

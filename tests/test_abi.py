@@ -173,6 +173,64 @@ def test_paged_decode_noalloc_host_validation(lib, kw, expect):
     assert rc == expect
 
 
+def _dec_checked(lib, ptrs=(1 << 20,) * 6, B=2, Hq=32, Hkv=8, d=128, bs=16, maxb=8, nblocks=100, splits=0):
+    q, kc, vc, bt, sl, o = ptrs
+    return lib.paged_attn_decode_checked(q, kc, vc, bt, sl, B, Hq, Hkv, d, bs, maxb, nblocks, splits, o, None)
+
+
+@pytest.mark.parametrize("kw,expect", [
+    (dict(nblocks=0), INVALID),                    # a pool needs at least one block
+    (dict(nblocks=-4), INVALID),
+    (dict(nblocks=1 << 27), UNSUPPORTED),          # token coordinates must fit in int32
+    (dict(maxb=1 << 27), UNSUPPORTED),
+    (dict(ptrs=(16, 16, None, 16, 16, 16)), INVALID),
+    (dict(d=80), UNSUPPORTED),
+    (dict(B=0, nblocks=0), OK),                    # empty batch: nothing to check
+])
+def test_paged_decode_checked_host_validation(lib, kw, expect):
+    assert _dec_checked(lib, **kw) == expect
+
+
+@pytest.mark.parametrize("kw,expect", [
+    (dict(nblocks=0), INVALID),
+    (dict(nblocks=1 << 27), UNSUPPORTED),
+    (dict(ks=-1.0), INVALID),
+    (dict(d=64), UNSUPPORTED),
+])
+def test_paged_decode_fp8_checked_host_validation(lib, kw, expect):
+    a = dict(ptrs=(1 << 20,) * 6, B=2, Hq=32, Hkv=8, d=128, bs=16, maxb=8, nblocks=100, splits=0, ks=0.5, vs=2.0)
+    a.update(kw)
+    q, kc, vc, bt, sl, o = a["ptrs"]
+    rc = lib.paged_attn_decode_fp8_checked(q, kc, vc, bt, sl, a["B"], a["Hq"], a["Hkv"], a["d"], a["bs"], a["maxb"],
+                                           a["nblocks"], a["splits"], ctypes.c_float(a["ks"]),
+                                           ctypes.c_float(a["vs"]), o, None)
+    assert rc == expect
+
+
+@pytest.mark.parametrize("kw,expect", [
+    (dict(nblocks=0), INVALID),
+    (dict(nblocks=1 << 27), UNSUPPORTED),
+    (dict(maxb=1 << 27), UNSUPPORTED),
+    (dict(scale=0.0), INVALID),
+    (dict(B=0), OK),
+])
+def test_paged_prefill_checked_host_validation(lib, kw, expect):
+    a = dict(ptrs=(1 << 20,) * 8, B=2, Hq=8, Hkv=2, d=128, bs=16, maxb=8, nblocks=100, max_q=32, total_q=40,
+             scale=0.088)
+    a.update(kw)
+    q, kc, vc, bt, sl, cq, o, lse = a["ptrs"]
+    rc = lib.paged_attn_prefill_checked(q, kc, vc, bt, sl, cq, a["B"], a["Hq"], a["Hkv"], a["d"], a["bs"], a["maxb"],
+                                        a["nblocks"], a["max_q"], a["total_q"], 1, ctypes.c_float(a["scale"]), o,
+                                        lse, None)
+    assert rc == expect
+
+
+def test_unchecked_paged_calls_reject_tables_wider_than_int32_positions(lib):
+    assert _dec(lib, maxb=1 << 27) == UNSUPPORTED
+    assert _chunked(lib, maxb=1 << 27) == UNSUPPORTED
+    assert _fp8(lib, maxb=1 << 27) == UNSUPPORTED
+
+
 def test_no_cpu_fallback_without_device(lib):
     """Valid arguments without a usable device fail loudly (no silent CPU path)."""
     import torch
@@ -183,6 +241,7 @@ def test_no_cpu_fallback_without_device(lib):
     assert _varlen(lib) < 0
     assert _chunked(lib) < 0
     assert _fp8(lib) < 0
+    assert _dec_checked(lib) < 0
     assert lib.attn_check_support(0) < 0
 
 

@@ -131,10 +131,14 @@ def test_mixed_rows_head_dim_64():
 
 def test_large_scores_scale_one():
     # |scores| up to ~100 (natural units): the row max of later tiles often
-    # exceeds the reference by more than 8 log2 units without any shaping
+    # exceeds the reference by more than 8 log2 units without any shaping.
+    # Such a softmax is peaked, so O is close to single rows of V; V is
+    # halved to keep |O| below 4, where rounding O to bf16 alone costs up to
+    # 2^-8 |O| <= 0.0156 of the 0.02 budget (the kernel is not the limit).
     spec = inputs.PrefillSpec(B=1, Hq=8, Hkv=2, T=640, S=640, d=128, causal=True, seed=83)
     q, k, v = inputs.make_prefill(spec)
     q = (q.float() * 2.0).to(torch.bfloat16)
+    v = (v.float() * 0.5).to(torch.bfloat16)
     assert np.abs(f64(q[0, :, 0]) @ f64(k[0, :, 0]).T).max() > 80.0
     _dense(q, k, v, True, 1.0, need_rows=50)
 

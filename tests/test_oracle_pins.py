@@ -364,3 +364,91 @@ def test_e4m3_decoder_hand_values_and_torch():
     codes = np.arange(256, dtype=np.uint8)
     ref = torch.from_numpy(codes).view(torch.float8_e4m3fn).to(torch.float64).numpy()
     np.testing.assert_array_equal(orc.decode_e4m3(codes), ref)
+
+
+# ---- pool bound and seq_len clamp (readings: an id outside the pool masks its
+# positions; a seq_len beyond the table row's capacity is clamped to it) ----
+
+def test_pool_bound_that_holds_every_id_changes_nothing():
+    q, kc, vc, table, lens, bs = _paged_case(60)
+    O1, L1 = orc.paged_decode(q, kc, vc, table, lens, bs, 0.3)
+    O2, L2 = orc.paged_decode(q, kc, vc, table, lens, bs, 0.3, num_blocks=kc.shape[0])
+    np.testing.assert_array_equal(O1, O2)
+    np.testing.assert_array_equal(L1, L2)
+
+
+def test_masked_blocks_equal_a_cache_without_them():
+    """Ids at or past num_blocks (and negative ones) drop their positions:
+    the result equals the decode over a new cache that holds only the other
+    positions, written out position by position into fresh blocks."""
+    q, kc, vc, table, lens, bs = _paged_case(61)
+    nb = kc.shape[0] // 2
+    t2 = table.copy()
+    t2[2, 1] = -5  # a negative id inside the sequence
+    O, L = orc.paged_decode(q, kc, vc, t2, lens, bs, 0.3, num_blocks=nb)
+    assert (t2[lens > 0] >= nb).any()  # some sequences lose blocks
+    for b in range(len(lens)):
+        keep = [p for p in range(int(lens[b])) if 0 <= t2[b, p // bs] < nb]
+        n = len(keep)
+        kb = np.zeros((max(1, -(-n // bs)), bs) + kc.shape[2:])
+        vb = np.zeros_like(kb)
+        for i, p in enumerate(keep):
+            kb[i // bs, i % bs] = kc[t2[b, p // bs], p % bs]
+            vb[i // bs, i % bs] = vc[t2[b, p // bs], p % bs]
+        tb = np.arange(kb.shape[0])[None]
+        Oc, Lc = orc.paged_decode(q[b:b + 1], kb, vb, tb, [n], bs, 0.3)
+        np.testing.assert_allclose(O[b], Oc[0], rtol=0, atol=1e-12)
+        np.testing.assert_allclose(L[b], Lc[0], rtol=0, atol=1e-12)
+        if n == 0:
+            assert np.all(O[b] == 0) and np.all(np.isneginf(L[b]))
+
+
+def test_seq_len_beyond_the_table_row_is_clamped():
+    q, kc, vc, table, lens, bs = _paged_case(62)
+    cap = table.shape[1] * bs
+    full = np.full_like(lens, cap)
+    t2 = np.where(table >= 0, table, 0)  # every entry a valid id
+    O1, L1 = orc.paged_decode(q, kc, vc, t2, full, bs, 0.3)
+    O2, L2 = orc.paged_decode(q, kc, vc, t2, full + 1000, bs, 0.3)
+    np.testing.assert_array_equal(O1, O2)
+    np.testing.assert_array_equal(L1, L2)
+    O3, L3 = orc.paged_decode(q, kc, vc, t2, -full, bs, 0.3)
+    assert np.all(O3 == 0) and np.all(np.isneginf(L3))
+
+
+def test_paged_prefill_with_masked_blocks_brute_force():
+    """Chunked prefill with some ids outside the pool, against a loop over
+    the positions in Python floats: row i of sequence b sits at position
+    L - T + i and sees the kept positions up to it."""
+    ctx, qlens = [9, 17, 30, 6], [4, 17, 3, 6]
+    q, kc, vc, table, lens, cu_q, bs = _chunked_case(63, ctx, qlens)
+    nb = kc.shape[0] - 4
+    t2 = table.copy()
+    t2[1, 2] = -1
+    t2[2, 0] = nb + 1
+    t2[3, :] = nb  # every block of sequence 3 outside the pool
+    lens = np.array(ctx)
+    lens[0] = 10 ** 6  # clamped to the row's capacity (10 blocks of 4)
+    t2[0, :10] = np.where(t2[0, :10] >= 0, t2[0, :10], 0)
+    for causal in (True, False):
+        O, L = orc.paged_prefill(q, kc, vc, t2, lens, cu_q, bs, 0.3, causal, num_blocks=nb)
+        Hq, Hkv = q.shape[1], kc.shape[2]
+        for b in range(len(ctx)):
+            S = min(max(int(lens[b]), 0), t2.shape[1] * bs)
+            T = int(cu_q[b + 1] - cu_q[b])
+            for i in range(T):
+                r = int(cu_q[b]) + i
+                for h in range(Hq):
+                    hk = h // (Hq // Hkv)
+                    ps = [p for p in range(S) if 0 <= t2[b, p // bs] < nb and (not causal or p <= S - T + i)]
+                    if not ps:
+                        assert np.all(O[r, h] == 0) and L[h, r] == -np.inf
+                        continue
+                    sc = [0.3 * sum(q[r, h, c] * kc[t2[b, p // bs], p % bs, hk, c] for c in range(q.shape[2]))
+                          for p in ps]
+                    m = max(sc)
+                    w = [math.exp(x - m) for x in sc]
+                    ref = [sum(wj * vc[t2[b, p // bs], p % bs, hk, c] for wj, p in zip(w, ps)) / sum(w)
+                           for c in range(q.shape[2])]
+                    np.testing.assert_allclose(O[r, h], ref, rtol=0, atol=1e-12)
+                    assert abs(L[h, r] - (m + math.log(sum(w)))) < 1e-12
