@@ -54,6 +54,33 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_tiled() {
   return fn;
 }
 
+// The prefill kernels move registers from warpgroup 2 to the softmax
+// warpgroups with setmaxnreg; the increase waits until the launch's
+// allocation can supply it, so every prefill kernel must have been compiled
+// with the per-thread count the split was sized for.  Checked once per
+// device, before any prefill is launched.
+bool prefill_registers_fit() {
+  const void* fns[] = {
+      reinterpret_cast<const void*>(prefill::prefill_fwd_sm100<64, prefill::kDense>),
+      reinterpret_cast<const void*>(prefill::prefill_fwd_sm100<128, prefill::kDense>),
+      reinterpret_cast<const void*>(prefill::prefill_fwd_sm100<64, prefill::kVarlen>),
+      reinterpret_cast<const void*>(prefill::prefill_fwd_sm100<128, prefill::kVarlen>),
+      reinterpret_cast<const void*>(prefill::prefill_fwd_sm100<64, prefill::kPaged>),
+      reinterpret_cast<const void*>(prefill::prefill_fwd_sm100<128, prefill::kPaged>),
+  };
+  for (const void* fn : fns) {
+    cudaFuncAttributes fa;
+    if (cudaFuncGetAttributes(&fa, fn) != cudaSuccess) {
+      cudaGetLastError();
+      return false;
+    }
+    const long long have = static_cast<long long>(fa.numRegs) * prefill::kThreads;
+    const long long need = 2LL * 128 * prefill::kSoftmaxRegs + 128LL * prefill::kOtherRegs;
+    if (have < need) return false;
+  }
+  return true;
+}
+
 // Probe a device once: sm_100 (compute capability 10.0) and a loadable image.
 int probe_device(int dev, DeviceState** out) {
   if (dev < 0 || dev >= kMaxDevices) return ATTN_ERR_INVALID_ARG;
@@ -73,6 +100,8 @@ int probe_device(int dev, DeviceState** out) {
       if (cudaFuncGetAttributes(&fa, prefill::prefill_fwd_sm100<128, prefill::kDense>) != cudaSuccess) {
         cudaGetLastError();
         st.status = ATTN_ERR_UNSUPPORTED;  // no sm_100a image for this device
+      } else if (!prefill_registers_fit()) {
+        st.status = ATTN_ERR_UNSUPPORTED;  // the prefill's register split would not fit its launch
       } else if (encode_tiled() == nullptr) {
         st.status = ATTN_ERR_CUDA;
       } else {

@@ -14,6 +14,8 @@
 //   warps 4-7  softmax for query tile 1
 //   warp  8    TMA producer (Q once, then a K ring and a V ring)
 //   warp  9    MMA issuer (one thread): S_t = Q_t K^T, O_t += P_t V
+//   warps 10-11 idle; with them the CTA is three whole warpgroups, so that
+//   warpgroup 2 can hand registers to the softmax warpgroups (setmaxnreg)
 // Tensor memory (512 columns x 128 lanes x 32 bit):
 //   S_0 cols [0,128), S_1 [128,256): fp32 scores; after the softmax the same
 //   columns hold P as packed bf16 (64 columns), the A operand of P V.
@@ -41,7 +43,17 @@ namespace prefill {
 
 constexpr int kBM = 128;               // rows per query tile (= TMEM lanes)
 constexpr int kBN = 128;               // keys per K/V tile
-constexpr int kThreads = 320;          // 10 warps
+constexpr int kThreads = 384;          // 12 warps: three warpgroups
+// Registers per thread after the split (setmaxnreg): the softmax warpgroups
+// hold a 128-score row per thread, warpgroup 2 (producer, MMA issuer, two
+// idle warps) needs few.  The kernel is compiled for 168 per thread at
+// launch (65536 / 384, in steps of 8); the split must not add up to more,
+// or the increase would wait forever -- the host checks the compiled count
+// before the first launch (kLaunchRegs).
+constexpr int kSoftmaxRegs = 216;
+constexpr int kOtherRegs = 72;
+constexpr int kLaunchRegs = 168;
+static_assert(2 * kSoftmaxRegs + kOtherRegs <= 3 * kLaunchRegs, "register split exceeds the launch allocation");
 constexpr int kWarpLoad = 8;
 constexpr int kWarpMma = 9;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
@@ -261,6 +273,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t tmem = sm.tmem_base;
   volatile int* abort_flag = &sm.abort_flag;
 
+  if (warp >= 8) {
+  // Warpgroup 2 (producer, MMA issuer, two idle warps) hands registers to
+  // the two softmax warpgroups, which hold a 128-score row per thread.
+  reg_dealloc<kOtherRegs>();
   if (warp == kWarpLoad) {
     // ------------------------------ producer ------------------------------
     // The whole warp runs the loop; lane 0 waits on the barriers.  Contiguous
@@ -448,7 +464,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       umma_commit(&sm.mma_done);
       mbar_wait_drain(&sm.mma_done, 0);
     }
+  }
   } else {
+    reg_alloc<kSoftmaxRegs>();
     // ------------------------------ softmax -------------------------------
     const int t = warp >> 2;              // query tile of this warpgroup
     const int r = threadIdx.x & 127;      // row within the tile = TMEM lane
