@@ -63,7 +63,11 @@ DEFAULT_WORKLOAD = "long"
 # bench reports null until a new capture replaces it.
 TRAFFIC = {
     # set: {"prefill": bytes per launch, "decode": bytes per call (split + combine), "csrc": hash}
-    "long": {"prefill": 489.93e6, "decode": 537.27e6 + 2.44e6, "csrc": "b98a9ce2d7f121e2"},
+    "long": {"prefill": 475.07e6, "decode": 539.56e6, "csrc": "613c7534a5d15138"},
+    "step": {"prefill": 12.65e6, "decode": 605.07e6, "csrc": "613c7534a5d15138"},
+    "fp8": {"prefill": 12.65e6, "decode": 306.13e6, "csrc": "613c7534a5d15138"},
+    "varlen": {"prefill": 343.58e6, "decode": 605.06e6, "csrc": "613c7534a5d15138"},
+    "chunked": {"prefill": 363.81e6, "decode": 605.11e6, "csrc": "613c7534a5d15138"},
 }
 
 
