@@ -246,22 +246,34 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int n0 = kv_tiles_for(m0, T, S, p.causal);
   const int n1 = kv_tiles_for(m0 + kBM, T, S, p.causal);
   const int n_max = max(n0, n1);
+  // The lead tile is the one with more key tiles (tile 1 of a causal block
+  // unless it lies past the end): its chain S -> softmax -> P V -> next S is
+  // the CTA's critical path, so its copies and MMAs go first.
+  const int lead = (n1 >= n0 && n1 > 0) ? 1 : 0;
 
-  // The first copies leave before the CTA-wide barrier: Q of both tiles and,
-  // for contiguous keys, K / V tile 0 (paged tiles need the warp's table reads).
+  // The first copies leave before the CTA-wide barrier, in the order the
+  // MMAs need them: Q of the lead tile, K tile 0, Q of the other tile, V
+  // tile 0 (K / V only for contiguous keys: paged tiles need the warp's
+  // table reads).
   const int pre = (MODE != kPaged && n_max > 0) ? 1 : 0;  // K / V tiles issued here
   if (warp == kWarpLoad && lane == 0) {
     const int nt[2] = {n0, n1};
-    for (int t = 0; t < 2; ++t) {
-      if (nt[t] == 0) continue;
+    auto load_q = [&](int t) {
+      if (nt[t] == 0) return;
       mbar_arrive_expect_tx(&sm.q_full[t], C::kTileBytes);
       for (int c = 0; c < C::kChunks; ++c)
         tma_load_4d(sm.q[t][c], &tmQ, &sm.q_full[t], c * 64, h, qoff + m0 + t * kBM, bc);
-    }
+    };
+    load_q(lead);
     if constexpr (MODE != kPaged) {
       if (pre) {
         mbar_arrive_expect_tx(&sm.k_full[0], C::kTileBytes);
         for (int c = 0; c < C::kChunks; ++c) tma_load_4d(sm.k[0][c], &tmK, &sm.k_full[0], c * 64, hk, koff, bc);
+      }
+    }
+    load_q(1 - lead);
+    if constexpr (MODE != kPaged) {
+      if (pre) {
         mbar_arrive_expect_tx(&sm.v_full[0], C::kTileBytes);
         for (int c = 0; c < C::kChunks; ++c) tma_load_4d(sm.v[0][c], &tmV, &sm.v_full[0], c * 64, hk, koff, bc);
       }
@@ -402,9 +414,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       constexpr uint32_t idesc_qk = make_idesc_bf16(kBM, kBN, 0, 0);  // Q, K both K-major
       constexpr uint32_t idesc_pv = make_idesc_bf16(kBM, D, 0, 1);    // P (TMEM), V MN-major
       const int nt[2] = {n0, n1};
+      const int ord[2] = {lead, 1 - lead};
       bool ok = true;
-      for (int t = 0; t < 2 && ok; ++t)
-        if (nt[t] > 0) ok = mbar_wait(&sm.q_full[t], 0, abort_flag);
 
       // O_t += P_t(jj) V(jj).  Every commit and every wait costs this thread
       // ~100 cycles on the critical path of a P hand-off, so V(jj) is waited
@@ -433,9 +444,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int s = j % C::kStages;
         if (!(ok = mbar_wait(&sm.k_full[s], (j / C::kStages) & 1, abort_flag))) break;
         tc_fence_after();
-        for (int t = 0; t < 2 && ok; ++t) {
+        for (int i = 0; i < 2 && ok; ++i) {
+          const int t = ord[i];
           // the previous P_t must be consumed before S_t is overwritten
-          if (j >= 1 && j - 1 < nt[t]) ok = issue_pv(t, j - 1, t == 0 || j - 1 >= nt[0], j == nt[t]);
+          if (j >= 1 && j - 1 < nt[t]) ok = issue_pv(t, j - 1, i == 0, j == nt[t]);
+          if (ok && j == 0 && nt[t] > 0) ok = mbar_wait(&sm.q_full[t], 0, abort_flag);
           if (ok && j < nt[t]) {
             const uint32_t tS = tmem + t * kBN;
             const uint32_t qbase = smem_u32(sm.q[t][0]);
@@ -455,8 +468,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       if (ok && n_max > 0) {
         const int jl = n_max - 1;
-        for (int t = 0; t < 2 && ok; ++t)
-          if (jl < nt[t]) ok = issue_pv(t, jl, t == 0 || jl >= nt[0], true);
+        for (int i = 0; i < 2 && ok; ++i)
+          if (jl < nt[ord[i]]) ok = issue_pv(ord[i], jl, i == 0, true);
 
       }
       // Every MMA issued above is complete once mma_done fires; after an
