@@ -63,11 +63,11 @@ DEFAULT_WORKLOAD = "long"
 # bench reports null until a new capture replaces it.
 TRAFFIC = {
     # set: {"prefill": bytes per launch, "decode": bytes per call (split + combine), "csrc": hash}
-    "long": {"prefill": 475.07e6, "decode": 539.56e6, "csrc": "613c7534a5d15138"},
-    "step": {"prefill": 12.65e6, "decode": 605.07e6, "csrc": "613c7534a5d15138"},
-    "fp8": {"prefill": 12.65e6, "decode": 306.13e6, "csrc": "613c7534a5d15138"},
-    "varlen": {"prefill": 343.58e6, "decode": 605.06e6, "csrc": "613c7534a5d15138"},
-    "chunked": {"prefill": 363.81e6, "decode": 605.11e6, "csrc": "613c7534a5d15138"},
+    "long": {"prefill": 478.92e6, "decode": 539.67e6, "csrc": "973c56d520211de5"},
+    "step": {"prefill": 12.65e6, "decode": 604.96e6, "csrc": "973c56d520211de5"},
+    "fp8": {"prefill": 12.65e6, "decode": 306.16e6, "csrc": "973c56d520211de5"},
+    "varlen": {"prefill": 334.97e6, "decode": 605.11e6, "csrc": "973c56d520211de5"},
+    "chunked": {"prefill": 362.45e6, "decode": 605.07e6, "csrc": "973c56d520211de5"},
 }
 
 
