@@ -262,20 +262,22 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (nt[t] == 0) return;
       mbar_arrive_expect_tx(&sm.q_full[t], C::kTileBytes);
       for (int c = 0; c < C::kChunks; ++c)
-        tma_load_4d(sm.q[t][c], &tmQ, &sm.q_full[t], c * 64, h, qoff + m0 + t * kBM, bc);
+        tma_load_4d_hint(sm.q[t][c], &tmQ, &sm.q_full[t], c * 64, h, qoff + m0 + t * kBM, bc, l2_policy_evict_first());
     };
     load_q(lead);
     if constexpr (MODE != kPaged) {
       if (pre) {
         mbar_arrive_expect_tx(&sm.k_full[0], C::kTileBytes);
-        for (int c = 0; c < C::kChunks; ++c) tma_load_4d(sm.k[0][c], &tmK, &sm.k_full[0], c * 64, hk, koff, bc);
+        for (int c = 0; c < C::kChunks; ++c)
+          tma_load_4d_hint(sm.k[0][c], &tmK, &sm.k_full[0], c * 64, hk, koff, bc, l2_policy_evict_last());
       }
     }
     load_q(1 - lead);
     if constexpr (MODE != kPaged) {
       if (pre) {
         mbar_arrive_expect_tx(&sm.v_full[0], C::kTileBytes);
-        for (int c = 0; c < C::kChunks; ++c) tma_load_4d(sm.v[0][c], &tmV, &sm.v_full[0], c * 64, hk, koff, bc);
+        for (int c = 0; c < C::kChunks; ++c)
+          tma_load_4d_hint(sm.v[0][c], &tmV, &sm.v_full[0], c * 64, hk, koff, bc, l2_policy_evict_last());
       }
     }
   }
@@ -298,6 +300,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // in one warp instruction instead of one after another.
     const int nt[2] = {n0, n1};
     int k_issued = pre, v_issued = pre;  // K / V tiles whose loads were issued
+    const uint64_t kv_pol = l2_policy_evict_last();  // K / V tiles are read again by the other heads and blocks
     bool tail_issued = false;
     constexpr int kBlocks = kBN / 16;     // 16-token blocks per tile
     const int cl = lane / kBlocks, il = lane % kBlocks;  // paged: this lane's (chunk, block)
@@ -339,14 +342,14 @@ __global__ void __launch_bounds__(kThreads, 1)
           mbar_arrive_expect_tx(&sm.k_full[s], tile_bytes);
           if constexpr (MODE != kPaged) {
             for (int c = 0; c < C::kChunks; ++c)
-              tma_load_4d(sm.k[s][c], &tmK, &sm.k_full[s], c * 64, hk, koff + j * kBN, bc);
+              tma_load_4d_hint(sm.k[s][c], &tmK, &sm.k_full[s], c * 64, hk, koff + j * kBN, bc, kv_pol);
           }
         }
       }
       if (!__shfl_sync(0xffffffffu, ok ? 1 : 0, 0)) break;
       if (my_copy)
-        tma_load_2d(reinterpret_cast<uint8_t*>(sm.k[s][cl]) + il * 16 * 128, &tmK, &sm.k_full[s],
-                    hk * D + cl * 64, my_id * 16);
+        tma_load_2d_hint(reinterpret_cast<uint8_t*>(sm.k[s][cl]) + il * 16 * 128, &tmK, &sm.k_full[s],
+                    hk * D + cl * 64, my_id * 16, kv_pol);
       if (lane == 0) {
         k_issued = j + 1;
         // V(j) reuses V(j - kStages)'s slot, freed by iteration j - kStages + 1
@@ -364,8 +367,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (lane == 0) mbar_arrive_expect_tx(&sm.v_tail, tile_bytes);
         __syncwarp();
         if (my_copy)
-          tma_load_2d(reinterpret_cast<uint8_t*>(sm.v[s][cl]) + il * 16 * 128, &tmV, &sm.v_tail,
-                      hk * D + cl * 64, my_id * 16);
+          tma_load_2d_hint(reinterpret_cast<uint8_t*>(sm.v[s][cl]) + il * 16 * 128, &tmV, &sm.v_tail,
+                      hk * D + cl * 64, my_id * 16, kv_pol);
         tail_issued = true;
         ok = __shfl_sync(0xffffffffu, mbar_wait(&sm.v_tail, 0, abort_flag) ? 1 : 0, 0) != 0;
         if (!ok) break;
@@ -388,13 +391,13 @@ __global__ void __launch_bounds__(kThreads, 1)
           mbar_arrive_expect_tx(&sm.v_full[s], tile_bytes);
           if constexpr (MODE != kPaged) {
             for (int c = 0; c < C::kChunks; ++c)
-              tma_load_4d(sm.v[s][c], &tmV, &sm.v_full[s], c * 64, hk, koff + j * kBN, bc);
+              tma_load_4d_hint(sm.v[s][c], &tmV, &sm.v_full[s], c * 64, hk, koff + j * kBN, bc, kv_pol);
           }
         }
         __syncwarp();
         if (my_copy)
-          tma_load_2d(reinterpret_cast<uint8_t*>(sm.v[s][cl]) + il * 16 * 128, &tmV, &sm.v_full[s],
-                      hk * D + cl * 64, my_id * 16);
+          tma_load_2d_hint(reinterpret_cast<uint8_t*>(sm.v[s][cl]) + il * 16 * 128, &tmV, &sm.v_full[s],
+                      hk * D + cl * 64, my_id * 16, kv_pol);
       }
       v_issued = j + 1;
     }
@@ -635,6 +638,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       __syncwarp();
       const int warp_row0 = t * kBM + (warp & 3) * 32;  // first row of this warp within the CTA's block
       const int chunk = lane % kChunksPerRow;
+      const uint64_t o_pol = l2_policy_evict_first();  // O is written once
 #pragma unroll 4
       for (int pass = 0; pass < 32 / kRowsPerPass; ++pass) {
         const int rl = pass * kRowsPerPass + lane / kChunksPerRow;  // row within the warp's 32
@@ -643,7 +647,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             *reinterpret_cast<const uint4*>(stage + rl * kRowBytes + ((chunk ^ (rl & (kChunksPerRow - 1))) * 16));
         if (rrow < T) {
           const size_t orow = VARLEN ? static_cast<size_t>(qoff) + rrow : static_cast<size_t>(b) * T + rrow;
-          reinterpret_cast<uint4*>(p.o + (orow * p.Hq + h) * D)[chunk] = val;
+          st_global_v4_hint(reinterpret_cast<uint4*>(p.o + (orow * p.Hq + h) * D) + chunk, val, o_pol);
         }
       }
     }
