@@ -32,6 +32,7 @@ from __future__ import annotations
 import argparse
 import hashlib
 import json
+import math
 import os
 import sys
 import threading
@@ -43,8 +44,9 @@ sys.path.insert(0, ROOT)
 METRIC = "prefill attn TFLOP/s & paged-decode KV GB/s, % of B200 roofline"
 UNIT = "% of 1xB200 roofline (summed over GPUs)"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
-PART_TIMING = ("each op alone: K back-to-back calls on the launching stream, CUDA events at the two ends, "
-               "right after the timed step loop")
+PART_MIN_MS = 20.0  # an op timed alone runs for at least this long (and at least K calls)
+PART_TIMING = ("each op alone: back-to-back calls on the launching stream (at least K, and at least "
+               f"{PART_MIN_MS:g} ms of them), CUDA events at the two ends, right after the timed step loop")
 
 WORKLOAD_SETS = {
     "long": ("long_prefill_16k", "long_decode_131k"),
@@ -533,9 +535,18 @@ def main():
     # event between two kernels would cut the programmatic overlap of one
     # kernel's prologue with the previous one's tail.
     ms_step, clocks = timed_region(torch, stream, step, K, sampler, world, dist)
-    # Each op alone, K back-to-back calls (the per-op roofline fractions).
-    ms_pre, clocks_pre = timed_region(torch, stream, lambda: pre.call(stream), K, sampler, world, dist)
-    ms_dec, clocks_dec = timed_region(torch, stream, lambda: decode_call(stream), K, sampler, world, dist)
+    # Each op alone (the per-op roofline fractions): at least K back-to-back
+    # calls and at least PART_MIN_MS of them, so that a short op is timed in
+    # steady state rather than over the first few calls after the step loop.
+    def part_calls(body):
+        t_est, _ = timed_region(torch, stream, body, 3, sampler, world, dist)
+        (n,) = dist_util.max_over_ranks([max(K, math.ceil(PART_MIN_MS / max(t_est, 1e-3)))], device=dev)
+        return int(n)
+
+    pre_body, dec_body = (lambda: pre.call(stream)), (lambda: decode_call(stream))
+    n_pre, n_dec = part_calls(pre_body), part_calls(dec_body)
+    ms_pre, clocks_pre = timed_region(torch, stream, pre_body, n_pre, sampler, world, dist)
+    ms_dec, clocks_dec = timed_region(torch, stream, dec_body, n_dec, sampler, world, dist)
     sampler.stop()
     status = fa.attn_read_device_status(clear=True)
     if status != 0:
@@ -599,10 +610,10 @@ def main():
     parts = {
         "prefill": {"op": pre.name, "ms": ms_pre, "tflops": pre_tflops, "peak": tpeak, "frac": pre_tflops / tpeak,
                     "peak_source": tpeak_src, "flops": flops, "algorithmic_bytes": pre.min_bytes,
-                    "traffic": pre_traffic, "traffic_note": pre_tnote, "clocks": clocks_pre},
+                    "traffic": pre_traffic, "traffic_note": pre_tnote, "calls": n_pre, "clocks": clocks_pre},
         "decode": {"op": dname, "ms": ms_dec, "gbs": dec_gbs, "peak": peaks["hbm_gbs"],
                    "frac": dec_gbs / peaks["hbm_gbs"], "peak_source": f"{peak_src} (hbm_gbs)", "bytes": dbytes,
-                   "traffic": dec_traffic, "traffic_note": dec_tnote, "clocks": clocks_dec},
+                   "traffic": dec_traffic, "traffic_note": dec_tnote, "calls": n_dec, "clocks": clocks_dec},
     }
     if ms_pre >= ms_dec:  # the op that takes longer alone
         roofline = {"bound": "tensor", "achieved": pre_tflops, "peak": tpeak, "unit": "TFLOP/s",
