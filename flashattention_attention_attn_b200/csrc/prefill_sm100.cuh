@@ -21,7 +21,12 @@
 //   columns hold P as packed bf16 (64 columns), the A operand of P V.
 //   O_0 [256, 256+D), O_1 [256+D, 256+2D): fp32 output accumulators.
 // The two query tiles ping-pong: while the softmax warps of one tile work,
-// the tensor core runs the other tile's MMAs.
+// the tensor core runs the other tile's MMAs.  The tile with more key tiles
+// (the lead) has its copies and, in every key iteration, its MMAs issued
+// first: its chain S -> softmax -> P V -> next S is the CTA's critical path.
+// K / V tiles are loaded with an L2 evict_last policy (the other heads of the
+// GQA group and the later query blocks read them again), Q and O with
+// evict_first.
 // The kernel is launched as a programmatic dependent of the previous grid on
 // the stream: barrier set-up, the tensor-memory allocation and (dense mode) L2
 // prefetches of the first tiles happen before the grid-dependency wait.  The
