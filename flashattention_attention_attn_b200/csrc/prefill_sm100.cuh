@@ -205,22 +205,41 @@ __global__ void __launch_bounds__(kThreads, 1)
   if constexpr (VARLEN) {
     if (p.items > 0) {
       // Compact grid: CTA -> work item blockIdx / Hq -> (sequence, query
-      // block) in the order of the full grid (top query blocks first,
-      // sequences ascending) but without the blocks past a sequence's end.
-      // Lane i holds sequence i's block count; every warp finds the same item.
+      // block), without the blocks past a sequence's end.  Packed prefill:
+      // the order of the full grid (top query blocks first, sequences
+      // ascending), so the heaviest blocks start first.  Lane i holds
+      // sequence i's block count; every warp finds the same item.
       const int len = (lane < p.B) ? p.cu_q[lane + 1] - p.cu_q[lane] : 0;
       const int nblocks = (len + 2 * kBM - 1) / (2 * kBM);
       int left = static_cast<int>(blockIdx.x) / p.Hq;
       b = -1;
-      for (int k = p.num_mblocks - 1; k >= 0 && b < 0; --k) {
-        uint32_t m = __ballot_sync(0xffffffffu, nblocks > k);
-        const int c = __popc(m);
-        if (left < c) {
-          for (int i = 0; i < left; ++i) m &= m - 1;  // drop the first `left` set bits
+      if constexpr (MODE == kPaged) {
+        // Chunked prefill: sequence-major (a sequence's query blocks, top
+        // first, are adjacent), so that its blocks read the same keys and
+        // values from L2 while they are there.
+        int incl = nblocks;  // inclusive prefix sum of the block counts
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+          const int y = __shfl_up_sync(0xffffffffu, incl, o);
+          if (lane >= o) incl += y;
+        }
+        const int excl = incl - nblocks;
+        const uint32_t m = __ballot_sync(0xffffffffu, left >= excl && left < incl);
+        if (m != 0) {
           b = __ffs(m) - 1;
-          mb = k;
-        } else {
-          left -= c;
+          mb = __shfl_sync(0xffffffffu, nblocks, b) - 1 - (left - __shfl_sync(0xffffffffu, excl, b));
+        }
+      } else {
+        for (int k = p.num_mblocks - 1; k >= 0 && b < 0; --k) {
+          uint32_t m = __ballot_sync(0xffffffffu, nblocks > k);
+          const int c = __popc(m);
+          if (left < c) {
+            for (int i = 0; i < left; ++i) m &= m - 1;  // drop the first `left` set bits
+            b = __ffs(m) - 1;
+            mb = k;
+          } else {
+            left -= c;
+          }
         }
       }
       if (b < 0) return;  // past the last item (the grid is an upper bound)
