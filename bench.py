@@ -65,11 +65,11 @@ DEFAULT_WORKLOAD = "long"
 # bench reports null until a new capture replaces it.
 TRAFFIC = {
     # set: {"prefill": bytes per launch, "decode": bytes per call (split + combine), "csrc": hash}
-    "long": {"prefill": 478.92e6, "decode": 539.67e6, "csrc": "973c56d520211de5"},
-    "step": {"prefill": 12.65e6, "decode": 604.96e6, "csrc": "973c56d520211de5"},
-    "fp8": {"prefill": 12.65e6, "decode": 306.16e6, "csrc": "973c56d520211de5"},
-    "varlen": {"prefill": 334.97e6, "decode": 605.11e6, "csrc": "973c56d520211de5"},
-    "chunked": {"prefill": 362.45e6, "decode": 605.07e6, "csrc": "973c56d520211de5"},
+    "long": {"prefill": 379.11e6, "decode": 539.69e6, "csrc": "4c546efed694eb30"},
+    "step": {"prefill": 12.65e6, "decode": 605.01e6, "csrc": "4c546efed694eb30"},
+    "fp8": {"prefill": 12.65e6, "decode": 306.32e6, "csrc": "4c546efed694eb30"},
+    "varlen": {"prefill": 277.57e6, "decode": 605.22e6, "csrc": "4c546efed694eb30"},
+    "chunked": {"prefill": 209.53e6, "decode": 605.28e6, "csrc": "4c546efed694eb30"},
 }
 
 
