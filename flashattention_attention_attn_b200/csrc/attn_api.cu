@@ -378,7 +378,7 @@ int auto_splits(int B, int groups, int max_blocks, int sms, int ctas_per_sm = 2)
 
 // The LSE merge, launched as a programmatic dependent of the split kernel so
 // that its launch and prologue overlap the split kernel's tail.  WPR warps
-// per (sequence, head) row: about 8 splits per warp, at most 16 warps.
+// per (sequence, head) row: about 8 splits per warp, at most 32 warps.
 template <int D, int WPR>
 int launch_combine_wpr(const decode::Params& p, const int32_t* lens, cudaStream_t stream) {
   using Shape = decode::CombineShape<WPR>;
@@ -412,7 +412,8 @@ int launch_combine(const decode::Params& p, const int32_t* lens, cudaStream_t st
   if (need <= 2) return launch_combine_wpr<D, 2>(p, lens, stream);
   if (need <= 4) return launch_combine_wpr<D, 4>(p, lens, stream);
   if (need <= 8) return launch_combine_wpr<D, 8>(p, lens, stream);
-  return launch_combine_wpr<D, 16>(p, lens, stream);
+  if (need <= 16) return launch_combine_wpr<D, 16>(p, lens, stream);
+  return launch_combine_wpr<D, 32>(p, lens, stream);
 }
 
 template <int D>

@@ -356,7 +356,7 @@ __global__ void __launch_bounds__((kKH + 1) * 32, 2)
 //   M = max_i lse_i,  O = sum_i e^{lse_i - M} o_i / sum_i e^{lse_i - M}.
 // WPR warps merge one (sequence, query head) row; a CTA holds
 // max(8, WPR) warps, i.e. max(1, 8 / WPR) rows, so that few splits give one
-// wave of CTAs and many splits spread each row over up to 16 warps.  Warp w
+// wave of CTAs and many splits spread each row over up to 32 warps.  Warp w
 // of a row takes splits w, w + WPR, ... with a running maximum (no separate
 // max pass) and kUnroll rows in flight per lane; lane c owns D/32
 // consecutive columns.  The row's warps are merged in shared memory in a
@@ -375,7 +375,7 @@ __global__ void __launch_bounds__(CombineShape<WPR>::kWarps * 32)
                 int num_splits, int chunk, int max_blocks) {
   using Shape = CombineShape<WPR>;
   constexpr int kPer = D / 32;
-  constexpr int kUnroll = (WPR == 1) ? 8 : 4;  // rows in flight per lane: one round for up to 8 splits
+  constexpr int kUnroll = 8;  // rows in flight per lane: one round for up to 8 splits per warp
   constexpr float kLog2e = 1.4426950408889634f;
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;

@@ -87,11 +87,13 @@ def test_garbage_past_sequence_end_is_ignored():
     check_close(f64(o), O, what="nan tail")
 
 
-@pytest.mark.parametrize("splits", [9, 17, 33, 65, 128])
-def test_many_splits_every_combine_shape(splits):
-    """Split counts that select 1, 2, 4, 8 and 16 warps per merged row."""
-    lens = [0, 5, 700, 2047, 2048, 1300, 16, 33]
-    spec = inputs.DecodeSpec(B=len(lens), Hq=32, Hkv=8, d=128, block_size=16, max_blocks=128, ctx_lo=0,
+@pytest.mark.parametrize("splits,max_blocks", [(9, 128), (17, 128), (33, 128), (65, 128), (128, 128),
+                                               (129, 320), (320, 320)])
+def test_many_splits_every_combine_shape(splits, max_blocks):
+    """Split counts that select 1, 2, 4, 8, 16 and 32 warps per merged row;
+    320 splits take a 32-warp row through two rounds of 8 splits per warp."""
+    lens = [0, 5, 700, 2047, 16 * max_blocks, 1300, 16, 33]
+    spec = inputs.DecodeSpec(B=len(lens), Hq=32, Hkv=8, d=128, block_size=16, max_blocks=max_blocks, ctx_lo=0,
                              ctx_hi=0, seed=16)
     inp = inputs.make_paged(spec, seq_lens=lens)
     o = run_decode(inp, num_splits=splits)
