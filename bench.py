@@ -65,11 +65,11 @@ DEFAULT_WORKLOAD = "long"
 # bench reports null until a new capture replaces it.
 TRAFFIC = {
     # set: {"prefill": bytes per launch, "decode": bytes per call (split + combine), "csrc": hash}
-    "long": {"prefill": 379.11e6, "decode": 539.69e6, "csrc": "4c546efed694eb30"},
-    "step": {"prefill": 12.65e6, "decode": 605.01e6, "csrc": "4c546efed694eb30"},
-    "fp8": {"prefill": 12.65e6, "decode": 306.32e6, "csrc": "4c546efed694eb30"},
-    "varlen": {"prefill": 277.57e6, "decode": 605.22e6, "csrc": "4c546efed694eb30"},
-    "chunked": {"prefill": 209.53e6, "decode": 605.28e6, "csrc": "4c546efed694eb30"},
+    "long": {"prefill": 383.36e6, "decode": 539.79e6, "csrc": "dd904f964a89aad4"},
+    "step": {"prefill": 12.65e6, "decode": 605.09e6, "csrc": "dd904f964a89aad4"},
+    "fp8": {"prefill": 12.65e6, "decode": 306.22e6, "csrc": "dd904f964a89aad4"},
+    "varlen": {"prefill": 279.27e6, "decode": 605.22e6, "csrc": "dd904f964a89aad4"},
+    "chunked": {"prefill": 209.80e6, "decode": 605.11e6, "csrc": "dd904f964a89aad4"},
 }
 
 
