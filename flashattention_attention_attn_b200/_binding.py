@@ -63,6 +63,11 @@ def library() -> ctypes.CDLL:
         lib.paged_attn_prefill_checked.argtypes = [vp, vp, vp, vp, vp, vp, c_int, c_int, c_int, c_int, c_int, c_int,
                                                    c_int, c_int, c_int, c_int, c_float, vp, vp, vp]
         lib.paged_attn_prefill_checked.restype = c_int
+        lib.paged_attn_decode_partial.argtypes = [vp, vp, vp, vp, vp, c_int, c_int, c_int, c_int, c_int, c_int,
+                                                  c_int, c_int, vp, vp, vp]
+        lib.paged_attn_decode_partial.restype = c_int
+        lib.attn_lse_merge.argtypes = [vp, vp, c_int, c_int, c_int, c_int, vp, vp]
+        lib.attn_lse_merge.restype = c_int
         lib.attn_check_support.argtypes = [c_int]
         lib.attn_check_support.restype = c_int
         lib.attn_status_string.argtypes = [c_int]
@@ -158,6 +163,26 @@ def paged_attn_decode_checked(q, k_cache, v_cache, block_table, seq_lens, B, Hq,
                                              _stream(stream))
     if rc != ATTN_OK:
         raise AttnError(rc, "paged_attn_decode_checked")
+
+
+def paged_attn_decode_partial(q, k_cache, v_cache, block_table, seq_lens, B, Hq, Hkv, d, block_size, max_blocks,
+                              num_blocks, num_splits, o_part, lse_part, stream=None) -> None:
+    """Decode over the keys held here, as fp32 o_part [B, Hq, d] and
+    lse_part [B, Hq] for a later attn_lse_merge (see attn.h)."""
+    rc = library().paged_attn_decode_partial(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_table),
+                                             _ptr(seq_lens), int(B), int(Hq), int(Hkv), int(d), int(block_size),
+                                             int(max_blocks), int(num_blocks), int(num_splits), _ptr(o_part),
+                                             _ptr(lse_part), _stream(stream))
+    if rc != ATTN_OK:
+        raise AttnError(rc, "paged_attn_decode_partial")
+
+
+def attn_lse_merge(o_parts, lse_parts, R, B, Hq, d, o, stream=None) -> None:
+    """Merge R partial results [R, B, Hq, d] / [R, B, Hq] into bf16 o [B, Hq, d] (see attn.h)."""
+    rc = library().attn_lse_merge(_ptr(o_parts), _ptr(lse_parts), int(R), int(B), int(Hq), int(d), _ptr(o),
+                                  _stream(stream))
+    if rc != ATTN_OK:
+        raise AttnError(rc, "attn_lse_merge")
 
 
 def paged_attn_decode_fp8_checked(q, k_cache, v_cache, block_table, seq_lens, B, Hq, Hkv, d, block_size, max_blocks,

@@ -379,8 +379,9 @@ int auto_splits(int B, int groups, int max_blocks, int sms, int ctas_per_sm = 2)
 // The LSE merge, launched as a programmatic dependent of the split kernel so
 // that its launch and prologue overlap the split kernel's tail.  WPR warps
 // per (sequence, head) row: about 8 splits per warp, at most 32 warps.
-template <int D, int WPR>
-int launch_combine_wpr(const decode::Params& p, const int32_t* lens, cudaStream_t stream) {
+template <int D, int WPR, bool kF32>
+int launch_combine_wpr(const decode::Params& p, const int32_t* lens, void* out, float* out_lse,
+                       cudaStream_t stream) {
   using Shape = decode::CombineShape<WPR>;
   const long long rows = static_cast<long long>(p.B) * p.Hq;
   cudaLaunchConfig_t cfg;
@@ -396,30 +397,34 @@ int launch_combine_wpr(const decode::Params& p, const int32_t* lens, cudaStream_
   cfg.numAttrs = 1;
   const float* po = p.part_o;
   const float* pl = p.part_lse;
-  if (cudaLaunchKernelEx(&cfg, decode::lse_combine<D, WPR>, po, pl, lens, p.o, p.B, p.Hq, p.num_splits,
-                         p.chunk, p.max_blocks) != cudaSuccess) {
+  if (cudaLaunchKernelEx(&cfg, decode::lse_combine<D, WPR, kF32>, po, pl, lens, out, out_lse, p.B, p.Hq,
+                         p.num_splits, p.chunk, p.max_blocks) != cudaSuccess) {
     cudaGetLastError();
     return ATTN_ERR_CUDA;
   }
   return ATTN_OK;
 }
 
-template <int D>
-int launch_combine(const decode::Params& p, const int32_t* lens, cudaStream_t stream) {
+// Merge p.num_splits partials per row into out: bf16 O, or (kF32) fp32 o
+// plus out_lse.  lens null: every partial of a row is merged.
+template <int D, bool kF32 = false>
+int launch_combine(const decode::Params& p, const int32_t* lens, void* out, float* out_lse, cudaStream_t stream) {
   const int per_warp = 8;
   const int need = (p.num_splits + per_warp - 1) / per_warp;
-  if (need <= 1) return launch_combine_wpr<D, 1>(p, lens, stream);
-  if (need <= 2) return launch_combine_wpr<D, 2>(p, lens, stream);
-  if (need <= 4) return launch_combine_wpr<D, 4>(p, lens, stream);
-  if (need <= 8) return launch_combine_wpr<D, 8>(p, lens, stream);
-  if (need <= 16) return launch_combine_wpr<D, 16>(p, lens, stream);
-  return launch_combine_wpr<D, 32>(p, lens, stream);
+  if (need <= 1) return launch_combine_wpr<D, 1, kF32>(p, lens, out, out_lse, stream);
+  if (need <= 2) return launch_combine_wpr<D, 2, kF32>(p, lens, out, out_lse, stream);
+  if (need <= 4) return launch_combine_wpr<D, 4, kF32>(p, lens, out, out_lse, stream);
+  if (need <= 8) return launch_combine_wpr<D, 8, kF32>(p, lens, out, out_lse, stream);
+  if (need <= 16) return launch_combine_wpr<D, 16, kF32>(p, lens, out, out_lse, stream);
+  return launch_combine_wpr<D, 32, kF32>(p, lens, out, out_lse, stream);
 }
 
+// o_part / lse_part non-null: the result is the partial (fp32 o [B, Hq, D],
+// natural-log lse [B, Hq]) over the keys this call sees, o unused.
 template <int D>
 int launch_decode(const void* q, const void* kc, const void* vc, const int32_t* table, const int32_t* lens, int B,
                   int Hq, int Hkv, int max_blocks, int num_blocks, int num_splits, void* o, cudaStream_t stream,
-                  const DeviceState* st) {
+                  const DeviceState* st, float* o_part = nullptr, float* lse_part = nullptr) {
   CUtensorMap mk, mv;
   if (make_map_decode_bf16(&mk, kc, Hkv, D, num_blocks) || make_map_decode_bf16(&mv, vc, Hkv, D, num_blocks))
     return ATTN_ERR_CUDA;
@@ -431,12 +436,13 @@ int launch_decode(const void* q, const void* kc, const void* vc, const int32_t* 
   if (num_splits > 65535 || groups > 65535 || B > 65535) return ATTN_ERR_UNSUPPORTED;
 
   decode::Params p;
+  const bool partial = o_part != nullptr;
   p.q = static_cast<const __nv_bfloat16*>(q);
   p.block_table = table;
   p.seq_lens = lens;
-  p.o = static_cast<__nv_bfloat16*>(o);
-  p.part_o = nullptr;
-  p.part_lse = nullptr;
+  p.o = partial ? nullptr : static_cast<__nv_bfloat16*>(o);
+  p.part_o = (partial && num_splits == 1) ? o_part : nullptr;  // a single split writes the partial itself
+  p.part_lse = (partial && num_splits == 1) ? lse_part : nullptr;
   p.B = B;
   p.Hq = Hq;
   p.Hkv = Hkv;
@@ -470,7 +476,9 @@ int launch_decode(const void* q, const void* kc, const void* vc, const int32_t* 
   dim3 grid(num_splits, groups, B);
   int rc = launch_pdl(decode::paged_decode_split<D>, grid, dim3((decode::kKH + 1) * 32), decode::smem_bytes<D>(),
                       stream, mk, mv, p);
-  if (rc == ATTN_OK && num_splits > 1) rc = launch_combine<D>(p, lens, stream);
+  if (rc == ATTN_OK && num_splits > 1)
+    rc = partial ? launch_combine<D, true>(p, lens, o_part, lse_part, stream)
+                 : launch_combine<D>(p, lens, o, nullptr, stream);
   if (ws != nullptr) cudaFreeAsync(ws, stream);
   return rc;
 }
@@ -527,7 +535,7 @@ int launch_decode_fp8(const void* q, const void* kc, const void* vc, const int32
   dim3 grid(num_splits, groups, B);
   int rc = launch_pdl(decode::paged_decode_split_fp8, grid, dim3((decode::kKH + 1) * 32), decode::smem_bytes_fp8(),
                       stream, mk, mv, p);
-  if (rc == ATTN_OK && num_splits > 1) rc = launch_combine<D>(p, lens, stream);
+  if (rc == ATTN_OK && num_splits > 1) rc = launch_combine<D>(p, lens, o, nullptr, stream);
   if (ws != nullptr) cudaFreeAsync(ws, stream);
   return rc;
 }
@@ -575,17 +583,22 @@ int decode_fp8_entry(const void* q, const void* k_cache, const void* v_cache, co
                            num_splits, k_scale, v_scale, o, stream, st);
 }
 
+// o_part / lse_part non-null: the partial form (o is then unused and may be null).
 int decode_entry(const void* q, const void* k_cache, const void* v_cache, const int32_t* block_table,
                  const int32_t* seq_lens, int B, int Hq, int Hkv, int d, int block_size, int max_blocks,
-                 int num_blocks, int num_splits, void* o, cudaStream_t stream) {
+                 int num_blocks, int num_splits, void* o, cudaStream_t stream, float* o_part = nullptr,
+                 float* lse_part = nullptr) {
   int rc = check_paged_common(B, Hq, Hkv, d, block_size, max_blocks, num_blocks);
   if (rc != ATTN_OK || B == 0) return rc;
+  const bool partial = o_part != nullptr || lse_part != nullptr;
   if (q == nullptr || k_cache == nullptr || v_cache == nullptr || block_table == nullptr || seq_lens == nullptr ||
-      o == nullptr)
+      (partial ? (o_part == nullptr || lse_part == nullptr) : o == nullptr))
     return ATTN_ERR_INVALID_ARG;
   if (d != 64 && d != 128) return ATTN_ERR_UNSUPPORTED;
   if (Hq / Hkv > 8) return ATTN_ERR_UNSUPPORTED;
-  if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(o)) return ATTN_ERR_UNSUPPORTED;
+  if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache)) return ATTN_ERR_UNSUPPORTED;
+  if (partial ? (!aligned16(o_part) || (reinterpret_cast<uintptr_t>(lse_part) & 3u)) : !aligned16(o))
+    return ATTN_ERR_UNSUPPORTED;
   if ((reinterpret_cast<uintptr_t>(block_table) & 3u) || (reinterpret_cast<uintptr_t>(seq_lens) & 3u))
     return ATTN_ERR_UNSUPPORTED;
   DeviceState* st = nullptr;
@@ -593,9 +606,42 @@ int decode_entry(const void* q, const void* k_cache, const void* v_cache, const 
   if (rc != ATTN_OK) return rc;
   if (d == 64)
     return launch_decode<64>(q, k_cache, v_cache, block_table, seq_lens, B, Hq, Hkv, max_blocks, num_blocks,
-                             num_splits, o, stream, st);
+                             num_splits, o, stream, st, o_part, lse_part);
   return launch_decode<128>(q, k_cache, v_cache, block_table, seq_lens, B, Hq, Hkv, max_blocks, num_blocks,
-                            num_splits, o, stream, st);
+                            num_splits, o, stream, st, o_part, lse_part);
+}
+
+// Merge R partials per (sequence, query head) row into bf16 O with the
+// decode's LSE combine kernel (every partial of a row taken).
+int lse_merge_entry(const float* o_parts, const float* lse_parts, int R, int B, int Hq, int d, void* o,
+                    cudaStream_t stream) {
+  if (R <= 0 || B < 0 || Hq <= 0 || d <= 0) return ATTN_ERR_INVALID_ARG;
+  if (B == 0) return ATTN_OK;
+  if (o_parts == nullptr || lse_parts == nullptr || o == nullptr) return ATTN_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return ATTN_ERR_UNSUPPORTED;
+  if (R > 65535 || static_cast<long long>(B) * Hq > (1LL << 30)) return ATTN_ERR_UNSUPPORTED;
+  if (!aligned16(o_parts) || !aligned16(o) || (reinterpret_cast<uintptr_t>(lse_parts) & 3u))
+    return ATTN_ERR_UNSUPPORTED;
+  DeviceState* st = nullptr;
+  int rc = current_device_state(&st);
+  if (rc != ATTN_OK) return rc;
+  decode::Params p;
+  p.q = nullptr;
+  p.block_table = nullptr;
+  p.seq_lens = nullptr;
+  p.o = static_cast<__nv_bfloat16*>(o);
+  p.part_o = const_cast<float*>(o_parts);
+  p.part_lse = const_cast<float*>(lse_parts);
+  p.B = B;
+  p.Hq = Hq;
+  p.Hkv = Hq;
+  p.max_blocks = 1;
+  p.num_blocks = 1;
+  p.num_splits = R;
+  p.chunk = 1;
+  p.scale_log2 = 1.0f;
+  if (d == 64) return launch_combine<64>(p, nullptr, o, nullptr, stream);
+  return launch_combine<128>(p, nullptr, o, nullptr, stream);
 }
 
 int prefill_paged_entry(const void* q, const void* k_cache, const void* v_cache, const int32_t* block_table,
@@ -735,6 +781,20 @@ extern "C" int paged_attn_decode_checked(const void* q, const void* k_cache, con
                                          void* o, attn_stream_t stream) {
   return decode_entry(q, k_cache, v_cache, block_table, seq_lens, B, Hq, Hkv, d, block_size, max_blocks,
                       num_blocks, num_splits, o, reinterpret_cast<cudaStream_t>(stream));
+}
+
+extern "C" int paged_attn_decode_partial(const void* q, const void* k_cache, const void* v_cache,
+                                         const int32_t* block_table, const int32_t* seq_lens, int B, int Hq, int Hkv,
+                                         int d, int block_size, int max_blocks, int num_blocks, int num_splits,
+                                         float* o_part, float* lse_part, attn_stream_t stream) {
+  if (o_part == nullptr || lse_part == nullptr) return ATTN_ERR_INVALID_ARG;
+  return decode_entry(q, k_cache, v_cache, block_table, seq_lens, B, Hq, Hkv, d, block_size, max_blocks,
+                      num_blocks, num_splits, nullptr, reinterpret_cast<cudaStream_t>(stream), o_part, lse_part);
+}
+
+extern "C" int attn_lse_merge(const float* o_parts, const float* lse_parts, int R, int B, int Hq, int d, void* o,
+                              attn_stream_t stream) {
+  return lse_merge_entry(o_parts, lse_parts, R, B, Hq, d, o, reinterpret_cast<cudaStream_t>(stream));
 }
 
 extern "C" int attn_check_support(int device) {
@@ -885,7 +945,7 @@ int launch_decode_noalloc(const void* q, const void* kc, const void* vc, const i
   dim3 grid(num_splits, groups, B);
   decode::paged_decode_split<D><<<grid, (decode::kKH + 1) * 32, decode::smem_bytes<D>(), stream>>>(mk, mv, p);
   int rc = launch_status();
-  if (rc == ATTN_OK && num_splits > 1) rc = launch_combine<D>(p, lens, stream);
+  if (rc == ATTN_OK && num_splits > 1) rc = launch_combine<D>(p, lens, o, nullptr, stream);
   return rc;
 }
 

@@ -68,8 +68,8 @@ struct Params {
   const __nv_bfloat16* q;      // [B, Hq, D]
   const int32_t* block_table;  // [B, max_blocks]
   const int32_t* seq_lens;     // [B]
-  __nv_bfloat16* o;            // [B, Hq, D] (written when num_splits == 1)
-  float* part_o;               // [num_splits, B, Hq, D]
+  __nv_bfloat16* o;            // [B, Hq, D]: written by a single split, or null (see part_o)
+  float* part_o;               // [num_splits, B, Hq, D]; a single split writes here when o is null
   float* part_lse;             // [num_splits, B, Hq]
   int B, Hq, Hkv, max_blocks;
   int num_blocks;              // pool size: block ids outside [0, num_blocks) are masked
@@ -129,12 +129,19 @@ __global__ void __launch_bounds__((kKH + 1) * 32, 2)
   const int blk1 = min(nb, blk0 + p.chunk);
   if (blk0 >= blk1) {
     // Empty range.  With several splits the combine skips it (and writes
-    // zeros for an empty sequence); with one split this CTA owns the output.
+    // zeros for an empty sequence); with one split this CTA owns the output:
+    // O = 0, or a partial o = 0 with lse = -inf.
     if (p.num_splits == 1 && L <= 0) {
       const int G = p.Hq / p.Hkv;
       const int heads = min(kKH, p.Hkv - hg * kKH) * G;
-      __nv_bfloat16* out = p.o + (static_cast<size_t>(b) * p.Hq + hg * kKH * G) * D;
-      for (int i = threadIdx.x; i < heads * D; i += blockDim.x) out[i] = __float2bfloat16_rn(0.f);
+      const size_t head0 = static_cast<size_t>(b) * p.Hq + hg * kKH * G;
+      if (p.o != nullptr) {
+        __nv_bfloat16* out = p.o + head0 * D;
+        for (int i = threadIdx.x; i < heads * D; i += blockDim.x) out[i] = __float2bfloat16_rn(0.f);
+      } else {
+        for (int i = threadIdx.x; i < heads * D; i += blockDim.x) p.part_o[head0 * D + i] = 0.f;
+        for (int i = threadIdx.x; i < heads; i += blockDim.x) p.part_lse[head0 + i] = -INFINITY;
+      }
     }
     return;
   }
@@ -317,7 +324,7 @@ __global__ void __launch_bounds__((kKH + 1) * 32, 2)
   const float inv0 = l0 > 0.f ? 1.0f / l0 : 0.f, inv1 = l1 > 0.f ? 1.0f / l1 : 0.f;
   const int g0 = 2 * quad, g1 = 2 * quad + 1;
   const size_t head0 = static_cast<size_t>(b) * p.Hq + hk * G;  // first query head of this kv head
-  if (p.num_splits == 1) {
+  if (p.num_splits == 1 && p.o != nullptr) {
 #pragma unroll
     for (int mm = 0; mm < D / 16; ++mm) {
       const int dd = mm * 16 + g_row;
@@ -362,17 +369,40 @@ __global__ void __launch_bounds__((kKH + 1) * 32, 2)
 // consecutive columns.  The row's warps are merged in shared memory in a
 // fixed order (deterministic).  Launched as a programmatic dependent of the
 // split kernel: everything before grid_dependency_wait() overlaps its tail.
+// kF32: write the merged row as fp32 o [B, Hq, D] plus its natural-log
+// lse [B, Hq] (itself a partial that a later merge can take), else as bf16.
+// seq_lens null: every one of the num_splits partials of a row is merged
+// (partials gathered from other devices; an empty one has lse = -inf).
 template <int WPR>
 struct CombineShape {
   static constexpr int kWarps = WPR > 8 ? WPR : 8;
   static constexpr int kRows = kWarps / WPR;
 };
 
-template <int D, int WPR>
+// One lane's kPer columns of a merged row: tot / ws, and the row's lse from
+// its log2-domain maximum M and weight sum ws (ws = 0: no key, o = 0, lse = -inf).
+template <int kPer, bool kF32>
+__device__ __forceinline__ void store_merged(void* out, float* out_lse, int row_id, int lane, const float* tot,
+                                             float M, float ws) {
+  constexpr int D = kPer * 32;
+  const float inv = ws > 0.f ? 1.0f / ws : 0.f;
+  if constexpr (kF32) {
+    float* dst = static_cast<float*>(out) + static_cast<size_t>(row_id) * D + lane * kPer;
+#pragma unroll
+    for (int e = 0; e < kPer; ++e) dst[e] = tot[e] * inv;
+    if (lane == 0) out_lse[row_id] = ws > 0.f ? (M + __log2f(ws)) * 0.69314718055994531f : -INFINITY;
+  } else {
+    __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(out) + static_cast<size_t>(row_id) * D + lane * kPer;
+#pragma unroll
+    for (int e = 0; e < kPer; ++e) dst[e] = __float2bfloat16_rn(tot[e] * inv);
+  }
+}
+
+template <int D, int WPR, bool kF32>
 __global__ void __launch_bounds__(CombineShape<WPR>::kWarps * 32)
     lse_combine(const float* __restrict__ part_o, const float* __restrict__ part_lse,
-                const int32_t* __restrict__ seq_lens, __nv_bfloat16* __restrict__ o, int B, int Hq,
-                int num_splits, int chunk, int max_blocks) {
+                const int32_t* __restrict__ seq_lens, void* __restrict__ out, float* __restrict__ out_lse, int B,
+                int Hq, int num_splits, int chunk, int max_blocks) {
   using Shape = CombineShape<WPR>;
   constexpr int kPer = D / 32;
   constexpr int kUnroll = 8;  // rows in flight per lane: one round for up to 8 splits per warp
@@ -389,7 +419,9 @@ __global__ void __launch_bounds__(CombineShape<WPR>::kWarps * 32)
   grid_dependency_wait();
   grid_launch_dependents();
   int nsp = 0;
-  if (live) {
+  if (live && seq_lens == nullptr) {
+    nsp = num_splits;
+  } else if (live) {
     const int L = checked_len(seq_lens, row_id / Hq, max_blocks, false);  // the split kernel reports
     nsp = min(num_splits, (((L + kBlock - 1) / kBlock) + chunk - 1) / chunk);  // splits holding data
   }
@@ -435,10 +467,7 @@ __global__ void __launch_bounds__(CombineShape<WPR>::kWarps * 32)
   }
   if constexpr (WPR == 1) {
     if (!live) return;
-    __nv_bfloat16* out = o + static_cast<size_t>(row_id) * D + lane * kPer;
-    const float inv = (wsum > 0.f) ? 1.0f / wsum : 0.f;  // no key at all: O = 0
-#pragma unroll
-    for (int e = 0; e < kPer; ++e) out[e] = __float2bfloat16_rn(acc[e] * inv);
+    store_merged<kPer, kF32>(out, out_lse, row_id, lane, acc, m, wsum);  // no key at all: O = 0
     return;
   } else {
 #pragma unroll
@@ -449,31 +478,25 @@ __global__ void __launch_bounds__(CombineShape<WPR>::kWarps * 32)
     }
     __syncthreads();
     if (!live || sub != 0) return;
-    __nv_bfloat16* out = o + static_cast<size_t>(row_id) * D + lane * kPer;
     // the first warp of the row merges its WPR warps
     const int w0 = local_row * WPR;
     float M = -INFINITY;
 #pragma unroll
     for (int w = 0; w < WPR; ++w) M = fmaxf(M, s_m[w0 + w]);
-    if (M == -INFINITY) {  // empty sequence, or no key inside the pool: O = 0
-#pragma unroll
-      for (int e = 0; e < kPer; ++e) out[e] = __float2bfloat16_rn(0.f);
-      return;
-    }
     float ws = 0.f;
     float tot[kPer];
 #pragma unroll
     for (int e = 0; e < kPer; ++e) tot[e] = 0.f;
+    if (M != -INFINITY) {  // else: empty sequence, or no key inside the pool: O = 0
 #pragma unroll
-    for (int w = 0; w < WPR; ++w) {
-      const float f = ex2_approx(s_m[w0 + w] - M);  // warps without rows: -inf -> 0
-      ws = fmaf(f, s_w[w0 + w], ws);
+      for (int w = 0; w < WPR; ++w) {
+        const float f = ex2_approx(s_m[w0 + w] - M);  // warps without rows: -inf -> 0
+        ws = fmaf(f, s_w[w0 + w], ws);
 #pragma unroll
-      for (int e = 0; e < kPer; ++e) tot[e] = fmaf(f, s_acc[w0 + w][lane * kPer + e], tot[e]);
+        for (int e = 0; e < kPer; ++e) tot[e] = fmaf(f, s_acc[w0 + w][lane * kPer + e], tot[e]);
+      }
     }
-    const float inv = 1.0f / ws;
-#pragma unroll
-    for (int e = 0; e < kPer; ++e) out[e] = __float2bfloat16_rn(tot[e] * inv);
+    store_merged<kPer, kF32>(out, out_lse, row_id, lane, tot, M, ws);
   }
 }
 

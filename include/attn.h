@@ -200,6 +200,67 @@ int paged_attn_decode_checked(const void* q, const void* k_cache, const void* v_
                               int num_blocks, int num_splits, void* o, attn_stream_t stream);
 
 /*
+ * paged_attn_decode_partial - the decode over part of each sequence's keys,
+ * returned in a form that other parts can be merged with.
+ *
+ * Context-parallel decode of long sequences: each device holds a contiguous
+ * range of every sequence's cached tokens in its own pool, with its own
+ * block table and lengths, and attends the query to that range only.  The
+ * per-range results are then merged (attn_lse_merge) after an exchange.  The
+ * split rests on the online-softmax statistics of the page "Snelle
+ * attention-kernels en operatorfusie versnellen AI-modellen" (the-ai.news),
+ * section "FlashAttention-type aandacht en gepagineerde aandacht": keys can
+ * be processed in any grouping as long as each group carries its maximum and
+ * sum; the natural-log LSE below carries both.
+ *
+ *   q, k_cache, v_cache, block_table, seq_lens, B, Hq, Hkv, d, block_size,
+ *   max_blocks, num_blocks, num_splits: as paged_attn_decode_checked, for
+ *                the keys this call sees (seq_lens[b] = the tokens of
+ *                sequence b held here; 0 allowed).
+ *   o_part       [B, Hq, d] fp32 (written): softmax-weighted average of the
+ *                values over the keys seen here, normalised by their own sum.
+ *   lse_part     [B, Hq] fp32 (written): ln sum_j exp(scale * <q, k_j>) over
+ *                those keys.  A query that sees no key gets o_part = 0 and
+ *                lse_part = -inf.
+ *
+ *   With every key of a sequence in one call, o_part equals the output of
+ *   paged_attn_decode before its rounding to bf16.
+ *   Supported and errors: as paged_attn_decode_checked; o_part 16-byte and
+ *   lse_part 4-byte aligned; ATTN_ERR_INVALID_ARG for a null o_part or
+ *   lse_part.  Workspace: as paged_attn_decode when num_splits resolves to
+ *   more than 1, none otherwise.
+ */
+int paged_attn_decode_partial(const void* q, const void* k_cache, const void* v_cache,
+                              const int32_t* block_table, const int32_t* seq_lens,
+                              int B, int Hq, int Hkv, int d, int block_size, int max_blocks,
+                              int num_blocks, int num_splits, float* o_part, float* lse_part,
+                              attn_stream_t stream);
+
+/*
+ * attn_lse_merge - merge R partial decode results of the same queries into
+ * the final output.
+ *
+ *   o_parts    [R, B, Hq, d] fp32, lse_parts [R, B, Hq] fp32: R results of
+ *              paged_attn_decode_partial over disjoint key ranges (for
+ *              instance one per device, gathered over NCCL).
+ *   o          [B, Hq, d] bf16 (written):
+ *                M = max_r lse_r,  w_r = exp(lse_r - M),
+ *                o = sum_r w_r o_r / sum_r w_r,
+ *              o = 0 where every lse_r is -inf.  This is the softmax over
+ *              the union of the key ranges, since sum_r w_r e^M is the sum
+ *              of exp of every score.  The result is deterministic (fixed
+ *              order, no atomics).
+ *
+ *   Supported: d in {64, 128}; 1 <= R <= 65535; o_parts and o 16-byte,
+ *   lse_parts 4-byte aligned; sm_100 device.  B == 0 is a no-op.
+ *   Errors: ATTN_ERR_INVALID_ARG for R <= 0, B < 0, Hq <= 0, d <= 0 or a
+ *   null pointer; ATTN_ERR_UNSUPPORTED otherwise outside the supported set;
+ *   ATTN_ERR_CUDA for a launch failure.  No workspace.
+ */
+int attn_lse_merge(const float* o_parts, const float* lse_parts, int R, int B, int Hq, int d, void* o,
+                   attn_stream_t stream);
+
+/*
  * attn_check_support - initialisation-time compatibility check of `device`,
  * in the spirit of the backend check at start-up described in the same
  * section of the page (an incompatible backend is reported as an error at

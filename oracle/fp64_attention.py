@@ -60,6 +60,7 @@ __all__ = [
     "paged_prefill",
     "decode_e4m3",
     "split_paged_decode",
+    "merge_partials",
 ]
 
 _ROW_GROUP = 256  # rows per numpy matrix product (memory bound only)
@@ -319,4 +320,33 @@ def split_paged_decode(q, k_cache, v_cache, block_table, seq_lens, block_size: i
         w = np.exp(pl - M[None, :])
         O[b] = (w[:, :, None] * po).sum(axis=0) / w.sum(axis=0)[:, None]
         LSE[b] = M + np.log(w.sum(axis=0))
+    return O, LSE
+
+
+def merge_partials(o_parts, lse_parts):
+    """Merge of R attention results over disjoint key sets of the same
+    queries, fp64.
+
+    o_parts [R, ..., d]: each result normalised by its own sum; lse_parts
+    [R, ...]: ln of that sum of exp of the scaled scores (-inf for a key set
+    that is empty for that query, whose o is then ignored).  Softmax over the
+    union of the sets, from the definition in the module docstring: with
+    M = max_r lse_r and w_r = exp(lse_r - M), the full sum of exp(s_j) is
+    e^M sum_r w_r and the full weighted value sum is e^M sum_r w_r o_r, so
+
+        O = sum_r w_r o_r / sum_r w_r,   LSE = M + ln sum_r w_r.
+
+    A query with every lse_r = -inf gets O = 0, LSE = -inf.  Returns
+    (O [..., d], LSE [...]).
+    """
+    po = np.asarray(o_parts, dtype=np.float64)
+    pl = np.asarray(lse_parts, dtype=np.float64)
+    M = pl.max(axis=0)
+    seen = np.isfinite(M)
+    Ms = np.where(seen, M, 0.0)
+    w = np.where(np.isneginf(pl), 0.0, np.exp(pl - Ms[None]))
+    wsum = w.sum(axis=0)
+    num = (w[..., None] * np.where(np.isneginf(pl)[..., None], 0.0, po)).sum(axis=0)
+    O = np.where(seen[..., None], num / np.where(seen, wsum, 1.0)[..., None], 0.0)
+    LSE = np.where(seen, Ms + np.log(np.where(seen, wsum, 1.0)), -np.inf)
     return O, LSE

@@ -33,7 +33,7 @@ def declared_functions():
 def test_header_declares_the_entry_points():
     names = declared_functions()
     for n in ("attn_fwd", "paged_attn_decode", "attn_check_support", "attn_status_string",
-              "attn_read_device_status"):
+              "attn_read_device_status", "paged_attn_decode_partial", "attn_lse_merge"):
         assert n in names
 
 
@@ -135,6 +135,47 @@ def _chunked(lib, ptrs=(1 << 20,) * 8, B=2, Hq=8, Hkv=2, d=128, bs=16, maxb=8, m
 ])
 def test_paged_prefill_host_validation(lib, kw, expect):
     assert _chunked(lib, **kw) == expect
+
+
+def _partial(lib, ptrs=(1 << 20,) * 7, B=2, Hq=32, Hkv=8, d=128, bs=16, maxb=8, nblk=64, splits=0):
+    q, kc, vc, bt, sl, op, lp = ptrs
+    return lib.paged_attn_decode_partial(q, kc, vc, bt, sl, B, Hq, Hkv, d, bs, maxb, nblk, splits, op, lp, None)
+
+
+@pytest.mark.parametrize("kw,expect", [
+    (dict(ptrs=(1 << 20,) * 5 + (None, 1 << 20)), INVALID),  # o_part
+    (dict(ptrs=(1 << 20,) * 6 + (None,)), INVALID),          # lse_part
+    (dict(ptrs=(None,) + (1 << 20,) * 6), INVALID),          # q
+    (dict(nblk=0), INVALID),
+    (dict(Hkv=6), INVALID),
+    (dict(d=96), UNSUPPORTED),
+    (dict(bs=8), UNSUPPORTED),
+    (dict(ptrs=(1 << 20,) * 5 + (8 + (1 << 20), 1 << 20)), UNSUPPORTED),  # o_part not 16-byte aligned
+    (dict(ptrs=(1 << 20,) * 6 + (2 + (1 << 20),)), UNSUPPORTED),          # lse_part not 4-byte aligned
+    (dict(B=0), OK),
+])
+def test_paged_decode_partial_host_validation(lib, kw, expect):
+    assert _partial(lib, **kw) == expect
+
+
+def _merge(lib, ptrs=(1 << 20,) * 3, R=2, B=2, Hq=8, d=128):
+    po, pl, o = ptrs
+    return lib.attn_lse_merge(po, pl, R, B, Hq, d, o, None)
+
+
+@pytest.mark.parametrize("kw,expect", [
+    (dict(R=0), INVALID),
+    (dict(Hq=0), INVALID),
+    (dict(B=-1), INVALID),
+    (dict(ptrs=(1 << 20, None, 1 << 20)), INVALID),
+    (dict(ptrs=(1 << 20, 1 << 20, None)), INVALID),
+    (dict(d=32), UNSUPPORTED),
+    (dict(R=70000), UNSUPPORTED),
+    (dict(ptrs=(4 + (1 << 20), 1 << 20, 1 << 20)), UNSUPPORTED),  # o_parts not 16-byte aligned
+    (dict(B=0), OK),
+])
+def test_lse_merge_host_validation(lib, kw, expect):
+    assert _merge(lib, **kw) == expect
 
 
 def _fp8(lib, ptrs=(1 << 20,) * 6, B=2, Hq=32, Hkv=8, d=128, bs=16, maxb=8, splits=0, ks=0.5, vs=2.0):

@@ -59,6 +59,22 @@ def _worker(rank, world, port, out_dir):
         dparts = [None] * world
         dist.all_gather_object(dparts, (lo, hi, Od, Ld))
 
+        # 5. context-parallel decode: every rank attends to its share of every
+        #    sequence, the partials are all-gathered (one collective) and merged
+        cinp = inputs.make_paged(inputs.DecodeSpec(B=4, Hq=8, Hkv=2, d=16, block_size=16, max_blocks=9, ctx_lo=0,
+                                                   ctx_hi=140, seed=23))
+        ctab, clens, _ = dist_util.context_shard(cinp.block_table, cinp.seq_lens, world, rank)
+        Oc, Lc = orc.paged_decode(f64(cinp.q), f64(cinp.k_cache), f64(cinp.v_cache), ctab.numpy(), clens.numpy(),
+                                  16, 0.25)
+        po, pl = dist_util.gather_partials(torch.from_numpy(Oc), torch.from_numpy(Lc))
+        assert po.shape == (world,) + Oc.shape and pl.shape == (world,) + Lc.shape
+        np.testing.assert_array_equal(po[rank].numpy(), Oc)
+        Om, Lm = orc.merge_partials(po.numpy(), pl.numpy())
+        Ofull, Lfull = orc.paged_decode(f64(cinp.q), f64(cinp.k_cache), f64(cinp.v_cache),
+                                        cinp.block_table.numpy(), cinp.seq_lens.numpy(), 16, 0.25)
+        np.testing.assert_allclose(Om, Ofull, rtol=0, atol=1e-12)
+        np.testing.assert_allclose(Lm, Lfull, rtol=0, atol=1e-12)
+
         if rank == 0:
             Of, Lf = orc.attention(f64(q), f64(k), f64(v), spec.scale, True)
             for qlo_, qhi_, O_, L_ in parts:
@@ -88,3 +104,23 @@ def test_shard_range_partitions(n, world):
         assert b == c and b >= a
     sizes = [b - a for a, b in spans]
     assert max(sizes) - min(sizes) <= 1
+
+
+@pytest.mark.parametrize("world", [1, 2, 3, 5, 8])
+def test_context_shares_cover_every_position_once(world):
+    lens = torch.tensor([0, 1, 15, 16, 17, 100, 160, 144, 999], dtype=torch.int32)  # 999: past the row, clamped
+    table = torch.arange(9 * 10, dtype=torch.int32).reshape(9, 10) * 7 + 3
+    seen = {b: [] for b in range(len(lens))}
+    for r in range(world):
+        t, n, lo = dist_util.context_shard(table, lens, world, r)
+        assert t.dtype == torch.int32 and n.dtype == torch.int32 and t.shape[0] == len(lens)
+        for b in range(len(lens)):
+            nb = (int(n[b]) + 15) // 16
+            assert torch.all(t[b, nb:] == -1)
+            for p in range(int(n[b])):  # local position p is global position lo*16 + p
+                g = int(lo[b]) * 16 + p
+                assert int(t[b, p // 16]) == int(table[b, g // 16]) and p % 16 == g % 16
+                seen[b].append(g)
+    for b in range(len(lens)):
+        L = min(int(lens[b]), 160)
+        assert sorted(seen[b]) == list(range(L)), b

@@ -261,6 +261,52 @@ def test_split_merge_equals_unsplit(splits):
     np.testing.assert_allclose(L2, L1, rtol=0, atol=1e-12)
 
 
+def test_merge_of_partials_closed_forms():
+    # two key sets with sums 1 and 3 (lse 0 and ln 3): weights 1/4 and 3/4, total sum 4
+    O, L = orc.merge_partials(np.array([[1.0, 0.0], [0.0, 1.0]]), np.array([0.0, math.log(3.0)]))
+    np.testing.assert_allclose(O, [0.25, 0.75], rtol=0, atol=1e-15)
+    assert abs(L - math.log(4.0)) < 1e-15
+    # an empty set (-inf) takes no part, whatever its o holds
+    O, L = orc.merge_partials(np.array([[np.nan, 7.0], [2.0, -1.0]]), np.array([-np.inf, 2.5]))
+    np.testing.assert_array_equal(O, [2.0, -1.0])
+    assert L == 2.5
+    # no key anywhere: O = 0, LSE = -inf
+    O, L = orc.merge_partials(np.ones((3, 4)), np.full(3, -np.inf))
+    assert np.all(O == 0) and np.isneginf(L)
+
+
+def _share_tables(table, lens, bs, cuts):
+    """Shares of every sequence cut at the given block boundaries (fractions
+    of its blocks), written position by position for the test."""
+    B, max_blocks = table.shape
+    shares = []
+    for r in range(len(cuts) - 1):
+        t = -np.ones((B, max_blocks), dtype=np.int32)
+        n = np.zeros(B, dtype=np.int64)
+        for b in range(B):
+            nb = (int(lens[b]) + bs - 1) // bs
+            lo, hi = int(cuts[r] * nb), int(cuts[r + 1] * nb)
+            t[b, :hi - lo] = table[b, lo:hi]
+            n[b] = max(0, min(int(lens[b]), hi * bs) - lo * bs)
+        shares.append((t, n))
+    return shares
+
+
+@pytest.mark.parametrize("cuts", [(0, 1), (0, 0.5, 1), (0, 0.2, 0.3, 1), (0, 0, 0.7, 0.7, 1)])
+def test_merge_of_context_shares_equals_unsplit_decode(cuts):
+    q, kc, vc, table, lens, bs = _paged_case(34)
+    O1, L1 = orc.paged_decode(q, kc, vc, table, lens, bs, 0.3)
+    parts = [orc.paged_decode(q, kc, vc, t, n, bs, 0.3) for t, n in _share_tables(table, lens, bs, cuts)]
+    assert sum(int(n.sum()) for _, n in _share_tables(table, lens, bs, cuts)) == int(lens.sum())
+    O2, L2 = orc.merge_partials(np.stack([o for o, _ in parts]), np.stack([lse for _, lse in parts]))
+    np.testing.assert_allclose(O2, O1, rtol=0, atol=1e-12)
+    np.testing.assert_allclose(L2, L1, rtol=0, atol=1e-12)
+    # the order of the parts does not matter
+    O3, L3 = orc.merge_partials(np.stack([o for o, _ in parts][::-1]), np.stack([lse for _, lse in parts][::-1]))
+    np.testing.assert_allclose(O3, O1, rtol=0, atol=1e-12)
+    np.testing.assert_allclose(L3, L1, rtol=0, atol=1e-12)
+
+
 def test_unused_table_entries_are_never_read():
     q, kc, vc, table, lens, bs = _paged_case(33)
     O1, L1 = orc.paged_decode(q, kc, vc, table, lens, bs, 0.3)
