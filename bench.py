@@ -65,11 +65,11 @@ DEFAULT_WORKLOAD = "long"
 # bench reports null until a new capture replaces it.
 TRAFFIC = {
     # set: {"prefill": bytes per launch, "decode": bytes per call (split + combine), "csrc": hash}
-    "long": {"prefill": 383.36e6, "decode": 539.79e6, "csrc": "dd904f964a89aad4"},
-    "step": {"prefill": 12.65e6, "decode": 605.09e6, "csrc": "dd904f964a89aad4"},
-    "fp8": {"prefill": 12.65e6, "decode": 306.22e6, "csrc": "dd904f964a89aad4"},
-    "varlen": {"prefill": 279.27e6, "decode": 605.22e6, "csrc": "dd904f964a89aad4"},
-    "chunked": {"prefill": 209.80e6, "decode": 605.11e6, "csrc": "dd904f964a89aad4"},
+    "long": {"prefill": 381.92e6, "decode": 539.75e6, "csrc": "c2db8360f1659fcb"},
+    "step": {"prefill": 12.65e6, "decode": 604.99e6, "csrc": "c2db8360f1659fcb"},
+    "fp8": {"prefill": 12.65e6, "decode": 306.29e6, "csrc": "c2db8360f1659fcb"},
+    "varlen": {"prefill": 279.62e6, "decode": 605.21e6, "csrc": "c2db8360f1659fcb"},
+    "chunked": {"prefill": 209.72e6, "decode": 605.10e6, "csrc": "c2db8360f1659fcb"},
 }
 
 
