@@ -34,6 +34,13 @@ int main(void) {
                 paged_attn_decode_fp8(p, p, p, (const int32_t*)p, (const int32_t*)p, 2, 32, 8, 128, 16, 8, 0,
                                       0.0f, 1.0f, p, NULL),
                 ATTN_ERR_INVALID_ARG);
+  /* context-parallel halves: a missing lse output, a merge of zero partials */
+  bad += expect("paged_attn_decode_partial null lse_part",
+                paged_attn_decode_partial(p, p, p, (const int32_t*)p, (const int32_t*)p, 2, 32, 8, 128, 16, 8, 64, 0,
+                                          (float*)p, NULL, NULL),
+                ATTN_ERR_INVALID_ARG);
+  bad += expect("attn_lse_merge R=0", attn_lse_merge((const float*)p, (const float*)p, 0, 2, 32, 128, p, NULL),
+                ATTN_ERR_INVALID_ARG);
   printf("attn_check_support(0) = %d (%s)\n", attn_check_support(0), attn_status_string(attn_check_support(0)));
   return bad;
 }
