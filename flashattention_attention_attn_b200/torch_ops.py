@@ -10,6 +10,9 @@ give output shapes without running anything) and with CUDA-graph capture.
     o = torch.ops.fa_b200.paged_attn_decode(q, k_cache, v_cache, block_table, seq_lens, num_splits)
     o = torch.ops.fa_b200.paged_attn_decode_fp8(q, k_cache, v_cache, block_table, seq_lens, num_splits,
                                                 k_scale, v_scale)
+    o_part, lse_part = torch.ops.fa_b200.paged_attn_decode_partial(q, k_cache, v_cache, block_table, seq_lens,
+                                                                   num_splits)
+    o = torch.ops.fa_b200.attn_lse_merge(o_parts, lse_parts)
 
 The op bodies only allocate the outputs and call the library on the current
 stream; there is no other path.  Shapes follow include/attn.h:
@@ -17,7 +20,10 @@ q [B,T,Hq,d], k/v [B,S,Hkv,d] -> o [B,T,Hq,d], lse [B,Hq,T];
 packed q [total_q,Hq,d], k/v [total_k,Hkv,d], cu_seqlens int32 [B+1]
 -> o [total_q,Hq,d], lse [Hq,total_q];
 decode q [B,Hq,d], caches [num_blocks,16,Hkv,d] (bf16, or e4m3 bytes),
-block_table [B,max_blocks], seq_lens [B] -> o [B,Hq,d].
+block_table [B,max_blocks], seq_lens [B] -> o [B,Hq,d];
+partial decode (the keys held here, the pool size read from the cache
+shape) -> o_part [B,Hq,d] fp32, lse_part [B,Hq] fp32; merge of R partials
+o_parts [R,B,Hq,d], lse_parts [R,B,Hq] -> o [B,Hq,d] bf16.
 """
 
 from __future__ import annotations
@@ -117,3 +123,38 @@ def paged_attn_decode_fp8(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch
 @paged_attn_decode_fp8.register_fake
 def _(q, k_cache, v_cache, block_table, seq_lens, num_splits, k_scale, v_scale):
     return torch.empty_like(q)
+
+
+@torch.library.custom_op("fa_b200::paged_attn_decode_partial", mutates_args=())
+def paged_attn_decode_partial(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor,
+                              block_table: torch.Tensor, seq_lens: torch.Tensor,
+                              num_splits: int) -> tuple[torch.Tensor, torch.Tensor]:
+    B, Hq, d = q.shape
+    num_blocks, block_size, Hkv = k_cache.shape[0], k_cache.shape[1], k_cache.shape[2]
+    o_part = torch.empty((B, Hq, d), device=q.device, dtype=torch.float32)
+    lse_part = torch.empty((B, Hq), device=q.device, dtype=torch.float32)
+    if B > 0:  # the entry point takes no empty outputs
+        _binding.paged_attn_decode_partial(q, k_cache, v_cache, block_table, seq_lens, B, Hq, Hkv, d, block_size,
+                                           block_table.shape[1], num_blocks, num_splits, o_part, lse_part,
+                                           torch.cuda.current_stream(q.device))
+    return o_part, lse_part
+
+
+@paged_attn_decode_partial.register_fake
+def _(q, k_cache, v_cache, block_table, seq_lens, num_splits):
+    B, Hq, _ = q.shape
+    return q.new_empty(q.shape, dtype=torch.float32), q.new_empty((B, Hq), dtype=torch.float32)
+
+
+@torch.library.custom_op("fa_b200::attn_lse_merge", mutates_args=())
+def attn_lse_merge(o_parts: torch.Tensor, lse_parts: torch.Tensor) -> torch.Tensor:
+    R, B, Hq, d = o_parts.shape
+    o = torch.empty((B, Hq, d), device=o_parts.device, dtype=torch.bfloat16)
+    if B > 0:
+        _binding.attn_lse_merge(o_parts, lse_parts, R, B, Hq, d, o, torch.cuda.current_stream(o_parts.device))
+    return o
+
+
+@attn_lse_merge.register_fake
+def _(o_parts, lse_parts):
+    return o_parts.new_empty(o_parts.shape[1:], dtype=torch.bfloat16)

@@ -37,6 +37,11 @@ def test_fake_shapes_without_running_anything():
         k8 = torch.empty(40, 16, 8, 128, dtype=torch.uint8)
         od = torch.ops.fa_b200.paged_attn_decode_fp8(qd, k8, k8, bt, torch.empty(5, dtype=torch.int32), 0, 0.5, 2.0)
         assert od.shape == qd.shape and od.dtype == torch.bfloat16
+        # context-parallel halves: fp32 partials, then the merge of R of them
+        op, lp = torch.ops.fa_b200.paged_attn_decode_partial(qd, kc, kc, bt, torch.empty(5, dtype=torch.int32), 0)
+        assert op.shape == qd.shape and op.dtype == torch.float32 and lp.shape == (5, 32) and lp.dtype == torch.float32
+        om = torch.ops.fa_b200.attn_lse_merge(torch.empty(3, 5, 32, 128), torch.empty(3, 5, 32))
+        assert om.shape == (5, 32, 128) and om.dtype == torch.bfloat16
 
 
 @pytest.mark.gpu
@@ -101,3 +106,33 @@ def test_packed_chunked_and_fp8_ops_match_the_oracle_and_the_binding():
                                                  din.v_scale)
     assert torch.equal(od.cpu(), od_ref)
     check_close(f64(od), oracle_decode_fp8(din)[0], what="torch op paged_attn_decode_fp8")
+
+
+@pytest.mark.gpu
+def test_context_parallel_ops_match_the_binding_and_the_oracle():
+    """Two shares of every sequence decoded with the partial op and merged
+    with the merge op inside torch.compile: identical to the direct binding
+    calls, and within the tolerance of the oracle's full decode."""
+    import flashattention_attention_attn_b200 as fa
+    from flashattention_attention_attn_b200 import dist_util
+    ds = inputs.DecodeSpec(B=4, Hq=32, Hkv=8, d=128, block_size=16, max_blocks=40, ctx_lo=0, ctx_hi=640, seed=65)
+    d = inputs.make_paged(ds)
+    dq, kc, vc = d.q.cuda(), d.k_cache.cuda(), d.v_cache.cuda()
+    shares = [dist_util.context_shard(d.block_table.cuda(), d.seq_lens.cuda(), 2, r)[:2] for r in range(2)]
+
+    def f(dq, kc, vc, t0, l0, t1, l1):
+        o0, s0 = torch.ops.fa_b200.paged_attn_decode_partial(dq, kc, vc, t0, l0, 0)
+        o1, s1 = torch.ops.fa_b200.paged_attn_decode_partial(dq, kc, vc, t1, l1, 0)
+        return torch.ops.fa_b200.attn_lse_merge(torch.stack([o0, o1]), torch.stack([s0, s1]))
+
+    g = torch.compile(f, backend="aot_eager", fullgraph=True)
+    o = g(dq, kc, vc, *shares[0], *shares[1])
+    po = torch.empty(2, 4, 32, 128, device="cuda")
+    pl = torch.empty(2, 4, 32, device="cuda")
+    for r, (t, n) in enumerate(shares):
+        fa.paged_attn_decode_partial(dq, kc, vc, t, n, 4, 32, 8, 128, 16, t.shape[1], kc.shape[0], 0, po[r], pl[r])
+    o_ref = torch.empty(4, 32, 128, device="cuda", dtype=torch.bfloat16)
+    fa.attn_lse_merge(po, pl, 2, 4, 32, 128, o_ref)
+    torch.cuda.synchronize()
+    assert torch.equal(o, o_ref)
+    check_close(f64(o), oracle_decode(d)[0], what="torch ops context-parallel decode")
