@@ -97,7 +97,8 @@ def gather_partials(o_part, lse_part, group=None):
 def context_parallel_decode(q, k_cache, v_cache, block_table, seq_lens, num_blocks: int, group=None,
                             num_splits: int = 0):
     """Context-parallel decode: q [B, Hq, d] bf16 replicated on every rank;
-    k_cache / v_cache [num_blocks, 16, Hkv, d] this rank's pool, block_table /
+    k_cache / v_cache [num_blocks, block_size, Hkv, d] this rank's pool (the
+    library takes 16-token blocks), block_table /
     seq_lens this rank's share of every sequence (for instance from
     context_shard).  Returns O [B, Hq, d] bf16, the same on every rank."""
     import torch
@@ -106,10 +107,10 @@ def context_parallel_decode(q, k_cache, v_cache, block_table, seq_lens, num_bloc
     from . import _binding
 
     B, Hq, d = q.shape
-    Hkv = k_cache.shape[2]
+    block_size, Hkv = k_cache.shape[1], k_cache.shape[2]
     o_part = torch.empty(B, Hq, d, device=q.device, dtype=torch.float32)
     lse_part = torch.empty(B, Hq, device=q.device, dtype=torch.float32)
-    _binding.paged_attn_decode_partial(q, k_cache, v_cache, block_table, seq_lens, B, Hq, Hkv, d, 16,
+    _binding.paged_attn_decode_partial(q, k_cache, v_cache, block_table, seq_lens, B, Hq, Hkv, d, block_size,
                                        block_table.shape[1], num_blocks, num_splits, o_part, lse_part)
     parts_o, parts_lse = gather_partials(o_part, lse_part, group)
     o = torch.empty(B, Hq, d, device=q.device, dtype=torch.bfloat16)
